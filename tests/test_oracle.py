@@ -1,0 +1,289 @@
+"""Pins of the float64 oracle against things other than itself (CPU only).
+
+Each group is chosen so that a plausible slip in the oracle (dropped scale, wrong
+causal direction, transposed operand, wrong log base, a missing term in the
+gradient, a wrong merge weight) fails at least one test.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import (attn_bwd, attn_fwd, attn_fwd_heads, lse_merge, ring_attention_blockwise,
+                    ring_attention_partials, ring_order)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# ---------------------------------------------------------------- brute force
+def _brute_fwd(q, k, v, causal, scale):
+    """Scalar triple loop, pure Python floats."""
+    S, Dh, Dv = len(q), len(q[0]), len(v[0])
+    O, L = [], []
+    for i in range(S):
+        s = []
+        for j in range(len(k)):
+            if causal and j > i:
+                continue
+            dot = 0.0
+            for d in range(Dh):
+                dot += q[i][d] * k[j][d]
+            s.append((j, dot * scale))
+        M = max(x for _, x in s)
+        Z = sum(math.exp(x - M) for _, x in s)
+        lse = M + math.log(Z)
+        o = [0.0] * Dv
+        for j, x in s:
+            w = math.exp(x - lse)
+            for d in range(Dv):
+                o[d] += w * v[j][d]
+        O.append(o)
+        L.append(lse)
+    return np.array(O), np.array(L)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S,Dh", [(1, 3), (7, 4), (13, 5)])
+def test_fwd_matches_brute_force(causal, S, Dh):
+    q, k, v = (_rand((S, Dh), s) * 1.5 for s in (1, 2, 3))
+    sc = 1.0 / math.sqrt(Dh)
+    Ob, Lb = _brute_fwd(q.tolist(), k.tolist(), v.tolist(), causal, sc)
+    O, L = attn_fwd(q, k, v, causal)
+    np.testing.assert_allclose(O, Ob, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(L, Lb, rtol=1e-12, atol=1e-12)
+
+
+def test_fwd_row_subset_and_chunking():
+    q, k, v = (_rand((40, 6), s) for s in (4, 5, 6))
+    O, L = attn_fwd(q, k, v, True)
+    rows = [39, 0, 17, 17, 3]
+    O2, L2 = attn_fwd(q, k, v, True, rows=rows, chunk=2)
+    np.testing.assert_allclose(O2, O[rows], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(L2, L[rows], rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("causal", [False, True])
+def test_identical_keys_give_mean_of_values(causal):
+    S, Dh = 11, 4
+    q, v = _rand((S, Dh), 7), _rand((S, Dh), 8)
+    kappa = _rand((Dh,), 9)
+    k = np.tile(kappa, (S, 1))
+    O, L = attn_fwd(q, k, v, causal)
+    sc = 1.0 / math.sqrt(Dh)
+    for i in range(S):
+        n = i + 1 if causal else S
+        np.testing.assert_allclose(O[i], v[:n].mean(axis=0), atol=1e-13)
+        assert abs(L[i] - (sc * q[i] @ kappa + math.log(n))) < 1e-13
+
+
+def test_one_hot_score_selects_one_value_row():
+    S, Dh = 9, 4
+    rng = np.random.default_rng(10)
+    k = rng.standard_normal((S, Dh)) * 0.01
+    J = 5
+    k[J] = np.array([60.0, 0, 0, 0])
+    q = np.tile(np.array([2.0, 0, 0, 0]), (S, 1))   # q . k_J * scale = 60
+    v = rng.standard_normal((S, Dh))
+    O, _ = attn_fwd(q, k, v, False)
+    np.testing.assert_allclose(O, np.tile(v[J], (S, 1)), atol=1e-15)
+
+
+def test_causal_row0_is_v0_and_lse_is_its_score():
+    S, Dh = 8, 16
+    q, k, v = (_rand((S, Dh), s) for s in (11, 12, 13))
+    O, L = attn_fwd(q, k, v, True)
+    np.testing.assert_allclose(O[0], v[0], atol=1e-15)
+    assert abs(L[0] - q[0] @ k[0] / 4.0) < 1e-14
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v_and_zero_q(causal):
+    S, Dh = 10, 8
+    q, k = _rand((S, Dh), 14), _rand((S, Dh), 15)
+    cvec = _rand((Dh,), 16)
+    O, _ = attn_fwd(q, k, np.tile(cvec, (S, 1)), causal)
+    np.testing.assert_allclose(O, np.tile(cvec, (S, 1)), atol=1e-14)
+    v = _rand((S, Dh), 17)
+    O, L = attn_fwd(np.zeros((S, Dh)), k, v, causal)
+    for i in range(S):
+        n = i + 1 if causal else S
+        np.testing.assert_allclose(O[i], v[:n].mean(axis=0), atol=1e-14)
+        assert abs(L[i] - math.log(n)) < 1e-14
+
+
+def test_explicit_scale_overrides_default():
+    q, k, v = (_rand((6, 4), s) for s in (18, 19, 20))
+    O1, L1 = attn_fwd(q, k, v, False, scale=0.3)
+    O2, L2 = attn_fwd(q * 0.3 / 0.5, k, v, False)  # default scale 1/sqrt(4) = 0.5
+    np.testing.assert_allclose(O1, O2, atol=1e-14)
+    np.testing.assert_allclose(L1, L2, atol=1e-14)
+
+
+# ---------------------------------------------------------------- backward
+def _loss(q, k, v, do, causal):
+    O, _ = attn_fwd(q, k, v, causal)
+    return float((O * do).sum())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_matches_central_finite_differences(causal):
+    S, Dh = 6, 3
+    q, k, v, do = (_rand((S, Dh), s) for s in (21, 22, 23, 24))
+    dq, dk, dv = attn_bwd(q, k, v, do, causal)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in itertools.product(range(S), range(Dh)):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            num[idx] = (_loss(args_p["q"], args_p["k"], args_p["v"], do, causal)
+                        - _loss(args_m["q"], args_m["k"], args_m["v"], do, causal)) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_matches_torch_float64_autograd(causal):
+    S, Dh = 33, 8
+    q, k, v, do = (_rand((S, Dh), s) for s in (25, 26, 27, 28))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    s = (tq @ tk.T) / math.sqrt(Dh)
+    if causal:
+        s = s.masked_fill(torch.ones(S, S, dtype=torch.bool).triu(1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ tv
+    o.backward(torch.tensor(do))
+    dq, dk, dv = attn_bwd(q, k, v, do, causal, chunk=7)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_column_sum_identities(causal):
+    """sum_j dK_j = 0 (each row of dS sums to zero) and sum_j dV_j = sum_i dO_i
+    (each row of P sums to one)."""
+    S, Dh = 40, 8
+    q, k, v, do = (_rand((S, Dh), s) for s in (29, 30, 31, 32))
+    dq, dk, dv = attn_bwd(q, k, v, do, causal)
+    np.testing.assert_allclose(dk.sum(axis=0), 0.0, atol=1e-12)
+    np.testing.assert_allclose(dv.sum(axis=0), do.sum(axis=0), atol=1e-12)
+
+
+# ---------------------------------------------------------------- merge
+def test_merge_single_part_is_identity_and_neg_inf_part_is_noop():
+    O = _rand((5, 4), 33)
+    L = _rand((5,), 34)
+    O1, L1 = lse_merge(O[None], L[None])
+    np.testing.assert_allclose(O1, O, atol=1e-15)
+    np.testing.assert_allclose(L1, L, atol=1e-15)
+    O2, L2 = lse_merge(np.stack([O, _rand((5, 4), 35)]), np.stack([L, np.full(5, -np.inf)]))
+    np.testing.assert_allclose(O2, O, atol=1e-15)
+    np.testing.assert_allclose(L2, L, atol=1e-15)
+
+
+def test_merge_all_neg_inf_gives_zero_and_neg_inf():
+    O, L = lse_merge(_rand((3, 2, 4), 36), np.full((3, 2), -np.inf))
+    assert np.all(O == 0.0) and np.all(np.isneginf(L))
+
+
+def test_merge_permutation_and_associativity():
+    Op, Lp = _rand((4, 6, 3), 37), _rand((4, 6), 38) * 3
+    O, L = lse_merge(Op, Lp)
+    perm = [2, 0, 3, 1]
+    Oq, Lq = lse_merge(Op[perm], Lp[perm])
+    np.testing.assert_allclose(Oq, O, atol=1e-14)
+    np.testing.assert_allclose(Lq, L, atol=1e-14)
+    Oa, La = lse_merge(Op[:2], Lp[:2])
+    Ob, Lb = lse_merge(np.stack([Oa, Op[2], Op[3]]), np.stack([La, Lp[2], Lp[3]]))
+    np.testing.assert_allclose(Ob, O, atol=1e-14)
+    np.testing.assert_allclose(Lb, L, atol=1e-14)
+
+
+def test_merge_of_key_halves_equals_full_attention():
+    S, Dh = 24, 8
+    q, k, v = (_rand((S, Dh), s) for s in (39, 40, 41))
+    O, L = attn_fwd(q, k, v, False)
+    parts = [attn_fwd(q, k[a:b], v[a:b], False) for a, b in ((0, 5), (5, 24))]
+    Om, Lm = lse_merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(Om, O, atol=1e-13)
+    np.testing.assert_allclose(Lm, L, atol=1e-13)
+
+
+# ---------------------------------------------------------------- ring algorithm
+def test_ring_order_matches_the_pages_worked_example():
+    rows = [tuple(int(x) for x in ln.split()) for ln in open(os.path.join(GOLDEN, "ring_walkthrough_d4.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    for dev, rnd, blk in rows:
+        assert ring_order(4, dev, False)[rnd - 1] == blk
+    for dev in range(4):  # after four rounds every device has used every block once
+        assert sorted(ring_order(4, dev, False)) == [0, 1, 2, 3]
+
+
+def test_ring_order_causal_drops_later_blocks():
+    assert ring_order(8, 0, True) == [0]
+    assert ring_order(8, 5, True) == [5, 4, 3, 2, 1, 0]
+    assert ring_order(8, 7, True) == [7, 6, 5, 4, 3, 2, 1, 0]
+    assert ring_order(8, 2, False) == [2, 1, 0, 7, 6, 5, 4, 3]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 6, 12])
+def test_blockwise_ring_equals_definition(causal, D):
+    S, Dh = 36, 8
+    q, k, v = (_rand((S, Dh), s) * 2 for s in (42, 43, 44))
+    O, L = attn_fwd(q, k, v, causal)
+    Ob, Lb = ring_attention_blockwise(q, k, v, D, causal)
+    np.testing.assert_allclose(Ob, O, atol=1e-12)
+    np.testing.assert_allclose(Lb, L, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blockwise_ring_is_order_independent(causal):
+    S, Dh, D = 32, 4, 8
+    q, k, v = (_rand((S, Dh), s) * 3 for s in (45, 46, 47))
+    O, L = attn_fwd(q, k, v, causal)
+    rng = np.random.default_rng(48)
+    reverse = [list(reversed(ring_order(D, r, causal))) for r in range(D)]
+    shuffled = [list(rng.permutation(ring_order(D, r, causal))) for r in range(D)]
+    for orders in (reverse, shuffled):
+        Ob, Lb = ring_attention_blockwise(q, k, v, D, causal, orders=orders)
+        np.testing.assert_allclose(Ob, O, atol=1e-12)
+        np.testing.assert_allclose(Lb, L, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_merged_ring_partials_equal_definition(causal):
+    S, Dh, D = 24, 8, 4
+    q, k, v = (_rand((S, Dh), s) for s in (49, 50, 51))
+    O, L = attn_fwd(q, k, v, causal)
+    Op, Lp = ring_attention_partials(q, k, v, D, causal)
+    Om, Lm = lse_merge(Op, Lp)
+    np.testing.assert_allclose(Om, O, atol=1e-12)
+    np.testing.assert_allclose(Lm, L, atol=1e-12)
+
+
+def test_uneven_split_is_rejected():
+    with pytest.raises(ValueError):
+        ring_attention_blockwise(np.zeros((10, 2)), np.zeros((10, 2)), np.zeros((10, 2)), 3, False)
+
+
+def test_heads_wrapper_accepts_bf16_torch_inputs():
+    from long_context_exact_fwd_b200.workloads import random_qkv
+    t = random_qkv(1, 2, 16, 8, seed=3)
+    O, L = attn_fwd_heads(t["q"], t["k"], t["v"], True)
+    O0, L0 = attn_fwd(t["q"][0, 1].double().numpy(), t["k"][0, 1].double().numpy(),
+                      t["v"][0, 1].double().numpy(), True)
+    np.testing.assert_allclose(O[0, 1], O0, atol=0)
+    np.testing.assert_allclose(L[0, 1], L0, atol=0)
