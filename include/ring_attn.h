@@ -1,0 +1,179 @@
+/*
+ * ring_attn.h -- C ABI of libringattn.so: exact ring attention on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (page: "精读笔记 · Ring Attention with Blockwise Transformers for
+ * Near-Infinite Context", §3.1-§3.5; page: "Ring Attention 与序列并行", conceptual
+ * pseudocode).  The S tokens of every (batch, head) are cut into D ring blocks of
+ * c = S / D tokens.  Query block r visits the key/value blocks in ring order -- at ring
+ * step t it works on block (r - t) mod D, step 0 being its own block -- and folds each
+ * block into a running max, running sum and rescaled accumulator (online softmax).  The
+ * result equals plain softmax(Q K^T * scale + mask) V with no approximation.  On one GPU
+ * the D positions are virtual: the same kernel processes all of them; no data moves
+ * between devices.
+ *
+ * Conventions shared by every entry point
+ *   Layout     all per-token tensors are dense row-major [B][H][S][Dh] (Dh contiguous);
+ *              LSE and the other per-row statistics are [B][H][S] float32.
+ *   Pointers   device pointers (cudaMalloc / torch CUDA memory) unless stated; tensors
+ *              read by TMA (q, k, v and the backward inputs) must be 16-byte aligned.
+ *              The caller owns every buffer; the library never allocates or frees device
+ *              memory and never synchronises, except ring_attn_device_status.
+ *   Stream     `stream` is a cudaStream_t (NULL = legacy default stream); all work is
+ *              enqueued on it.  Calls return as soon as the work is enqueued.
+ *   Mask       causal != 0 selects the autoregressive mask on global positions: key j is
+ *              visible to query i iff j <= i.  The pages never state a mask; this is the
+ *              standard reading.  causal == 0 lets every query see every key.
+ *   Scale      scores are q.k * scale with scale = 1/sqrt(Dh) unless an _ex call passes
+ *              scale > 0.
+ *   LSE        natural log of sum_j exp(score_ij) over visible keys, float32.
+ *   Errors     every call returns RA_OK (0) or one of the RA_ERR_* codes below and never
+ *              throws; argument errors are detected before anything is enqueued.  A
+ *              device-side fault surfaces at the caller's next synchronisation.  A kernel
+ *              whose internal bounded wait expired leaves RA_ERR_TIMEOUT in the device
+ *              status word, read by ring_attn_device_status.
+ */
+#ifndef RING_ATTN_H_
+#define RING_ATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define RA_API __attribute__((visibility("default")))
+#else
+#define RA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  RA_OK = 0,
+  RA_ERR_ARG = 1,         /* null pointer, non-positive size, unknown dtype            */
+  RA_ERR_SHAPE = 2,       /* S % D != 0, unsupported Dh, or a size that overflows       */
+  RA_ERR_ALIGN = 3,       /* a TMA-read pointer is not 16-byte aligned                 */
+  RA_ERR_WORKSPACE = 4,   /* backward workspace null or smaller than required          */
+  RA_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed                      */
+  RA_ERR_TIMEOUT = 6,     /* a kernel gave up on a bounded internal wait               */
+  RA_ERR_DEVICE = 7       /* the current device is not compute capability 10.0         */
+};
+
+typedef enum { RA_BF16 = 0, RA_F32 = 1 } ra_dtype;
+
+/* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA headers. */
+typedef void* ra_stream;
+
+/*
+ * ring_attn_fwd -- forward pass, bf16 inputs (page "精读笔记 ...", §3.1 and §3.5 Algorithm 1).
+ *   q, k, v  [B][H][S][Dh] bf16, read only, 16-byte aligned.
+ *   o        [B][H][S][Dh] bf16, written: O = softmax(q k^T / sqrt(Dh) + mask) v, fp32
+ *            accumulated and rounded to nearest even once.
+ *   lse      [B][H][S] float32, written: the row log-sum-exp (natural log).
+ *   B, H, S  >= 1.  S need not be a multiple of the kernel's 128-row tiles.
+ *   Dh       head dimension; 128 on this path (else RA_ERR_SHAPE).
+ *   D        number of ring blocks, 1 <= D <= S and S % D == 0 (the pages' even split,
+ *            "limitations" paragraph of the close reading), else RA_ERR_SHAPE.
+ *   causal   0 or 1 (see Mask above).
+ * The result does not depend on D (order independence, §3.1); D fixes the order in which
+ * each query tile visits the key/value tiles.
+ */
+RA_API int ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
+                  int Dh, int D, int causal, ra_stream stream);
+
+/*
+ * ring_attn_fwd_ex -- forward pass with an explicit input dtype and scale.
+ *   dtype RA_BF16: as ring_attn_fwd (o is bf16).
+ *   dtype RA_F32 : q, k, v and o are float32; scores, exponentials and the accumulator are
+ *                  float32 on CUDA cores (no tensor-core rounding), any Dh in 1..256.
+ *   scale > 0 overrides 1/sqrt(Dh); scale <= 0 keeps the default.
+ */
+RA_API int ring_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
+                     int Dh, int D, int causal, ra_dtype dtype, float scale, ra_stream stream);
+
+/*
+ * ring_attn_bwd_workspace_size -- bytes of device workspace ring_attn_bwd needs:
+ * a float32 dQ accumulator [B][H][S][Dh] and a float32 row statistic [B][H][S] (Delta),
+ * each 256-byte aligned.  Returns 0 for invalid sizes.
+ */
+RA_API size_t ring_attn_bwd_workspace_size(int B, int H, int S, int Dh);
+
+/*
+ * ring_attn_bwd -- backward pass of ring_attn_fwd (bf16).  The pages state that training runs
+ * through the same blockwise ring structure but give no formulas; this is the analytic
+ * softmax gradient, with P recomputed from the saved LSE:
+ *   P = exp(q k^T * scale - lse), dV = P^T dO, dP = dO V^T, Delta = rowsum(dO * O),
+ *   dS = P * (dP - Delta), dQ = scale * dS K, dK = scale * dS^T Q.
+ *   q, k, v, o, dO : [B][H][S][Dh] bf16, read only, 16-byte aligned (o from ring_attn_fwd).
+ *   lse            : [B][H][S] float32 from ring_attn_fwd.
+ *   dq, dk, dv     : [B][H][S][Dh] bf16, written (fully overwritten).
+ *   workspace      : >= ring_attn_bwd_workspace_size(B, H, S, Dh) bytes of device memory,
+ *                    256-byte aligned; its contents on entry are ignored (it is cleared
+ *                    on the stream) and undefined on return.
+ *   Other arguments as ring_attn_fwd.  Each key/value tile visits the query tiles that
+ *   can see it, in ring order.
+ */
+RA_API int ring_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D, int causal, void* workspace,
+                  size_t workspace_bytes, ra_stream stream);
+
+/*
+ * ring_attn_merge -- combine P normalised partial outputs through their log-sum-exp
+ * (page "精读笔记 ...", §3.1: blocks may be combined in any order when their statistics are
+ * combined with rescaling; page "RingAttention large-context attention", 架构与算法: the
+ * partial outputs are aggregated into the final output).
+ *   o_parts   [P][B][H][S][Dh] float32, partial p normalised by its own softmax sum.
+ *   lse_parts [P][B][H][S] float32; -inf marks a partial with no visible key (weight 0).
+ *   o         [B][H][S][Dh] bf16, written: sum_p exp(lse_p - lse) * o_p.
+ *   lse       [B][H][S] float32, written: log(sum_p exp(lse_p)); -inf (and o = 0) when every
+ *             partial is -inf.
+ *   P >= 1, Dh % 4 == 0 and Dh <= 256, pointers 16-byte aligned.
+ */
+RA_API int ring_attn_merge(const float* o_parts, const float* lse_parts, int P, void* o, float* lse, int B, int H, int S,
+                    int Dh, ra_stream stream);
+
+/* ring_attn_merge_ex -- as ring_attn_merge with o of type out_dtype (RA_BF16 or RA_F32). */
+RA_API int ring_attn_merge_ex(const float* o_parts, const float* lse_parts, int P, void* o, float* lse, int B, int H,
+                       int S, int Dh, ra_dtype out_dtype, ra_stream stream);
+
+/*
+ * ring_attn_ring_order -- host only, no GPU needed.  Writes to blocks[0..n) the key/value
+ * blocks ring position r visits, in order: block (r - t) mod D at step t = 0..D-1 (page
+ * "精读笔记 ...", §3.5 4-device walk-through), dropping blocks j > r when causal.
+ * Returns n (>= 1), or -RA_ERR_ARG for bad arguments or max_blocks < n.
+ */
+RA_API int ring_attn_ring_order(int D, int r, int causal, int* blocks, int max_blocks);
+
+/*
+ * ring_attn_visit_tiles -- host only.  The exact sequence of 128-key tiles the forward
+ * kernel visits for the query tile of `tile_rows` rows starting at row q0: ring steps of
+ * the query tile's block, each step's tiles (those whose first key lies in that block)
+ * ascending, tiles wholly above the causal diagonal dropped.  Writes the tile indices to
+ * tiles[0..n) and returns n, or -RA_ERR_ARG.
+ */
+RA_API int ring_attn_visit_tiles(int S, int D, int causal, int q0, int tile_rows, int* tiles, int max_tiles);
+
+/*
+ * ring_attn_device_status -- synchronises `stream`, returns the device status word
+ * (RA_OK or the first RA_ERR_TIMEOUT a kernel recorded) and clears it.  Returns
+ * RA_ERR_CUDA if the synchronisation itself fails.
+ */
+RA_API int ring_attn_device_status(ra_stream stream);
+
+/*
+ * ring_attn_last_cuda_error -- diagnostics for RA_ERR_CUDA: the cudaError_t / CUresult value
+ * of the last failing CUDA call made by this library on the calling host thread (0 if none),
+ * and, when `site` is not NULL, a static string naming that call.
+ */
+RA_API int ring_attn_last_cuda_error(const char** site);
+
+/* Static English text for a status code. */
+RA_API const char* ring_attn_strerror(int code);
+
+/* Library ABI version (major * 100 + minor). */
+RA_API int ring_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RING_ATTN_H_ */

@@ -1,0 +1,313 @@
+// C ABI of libringattn.so: argument validation, TMA descriptor construction and kernel
+// launches on the caller's stream.  See include/ring_attn.h for the contract of every
+// entry point.  No device memory is allocated here and nothing synchronises except
+// ring_attn_device_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ring_attn.h"
+#include "fwd_sm100.cuh"
+#include "fwd_f32.cuh"
+#include "merge.cuh"
+#include "bwd_sm100.cuh"
+
+namespace {
+
+// Last failing CUDA call of this host thread (diagnostics for RA_ERR_CUDA).
+thread_local int g_last_cuda_code = 0;
+thread_local const char* g_last_cuda_site = "";
+
+int cuda_fail(int code, const char* site) {
+  g_last_cuda_code = code;
+  g_last_cuda_site = site;
+  return RA_ERR_CUDA;
+}
+
+constexpr int RA_VERSION = 100;
+constexpr int MAX_DEVICES = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DevInfo {
+  int sm_count = 0;
+  bool ok = false;          // compute capability 10.0
+  bool fwd_attr[2] = {false, false};
+  bool bwd_attr = false;
+};
+
+std::mutex g_dev_mu;
+DevInfo g_dev[MAX_DEVICES];
+bool g_dev_init[MAX_DEVICES] = {};
+
+// Current device's info (cached); nullptr on a CUDA failure.
+DevInfo* dev_info(int* status) {
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+    *status = cuda_fail(static_cast<int>(e), "cudaGetDevice");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev_init[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      *status = RA_ERR_CUDA;
+      return nullptr;
+    }
+    g_dev[dev].sm_count = sms;
+    g_dev[dev].ok = (major == 10 && minor == 0);
+    g_dev_init[dev] = true;
+  }
+  if (!g_dev[dev].ok) {
+    *status = RA_ERR_DEVICE;
+    return nullptr;
+  }
+  *status = RA_OK;
+  return &g_dev[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D tensor map over a [BH][S][Dh] bf16 tensor: box = 64 columns (128 B) x `box_rows` rows
+// x 1 head, 128-byte swizzle, zero fill outside [0, S) so tiles never read the next head.
+int make_map(CUtensorMap* map, const void* base, long long BH, int S, int Dh, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cuda_fail(-1, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Dh), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Dh) * 2, static_cast<cuuint64_t>(S) * Dh * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RA_OK : cuda_fail(static_cast<int>(r), "cuTensorMapEncodeTiled");
+}
+
+// Common shape checks.  Sizes are bounded so that every element index fits in int64 and
+// every per-head row index fits in int.
+int check_shape(int B, int H, int S, int Dh, int D) {
+  if (B <= 0 || H <= 0 || S <= 0 || Dh <= 0 || D <= 0) return RA_ERR_ARG;
+  if (D > S || S % D != 0) return RA_ERR_SHAPE;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > INT_MAX / 2) return RA_ERR_SHAPE;
+  if (static_cast<double>(BH) * S * Dh > 9.0e18 / 4) return RA_ERR_SHAPE;
+  return RA_OK;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RA_OK : cuda_fail(static_cast<int>(e), "kernel launch");
+}
+
+template <int HD>
+int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D, int causal,
+             float scale, cudaStream_t stream) {
+  using namespace ra::fwd;
+  int st = RA_OK;
+  DevInfo* di = dev_info(&st);
+  if (!di) return st;
+  const long long BH = static_cast<long long>(B) * H;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, BH, S, HD, BM)) != RA_OK) return st;
+  if ((st = make_map(&mk, k, BH, S, HD, BN)) != RA_OK) return st;
+  if ((st = make_map(&mv, v, BH, S, HD, BN)) != RA_OK) return st;
+  Params p;
+  p.BH = static_cast<int>(BH);
+  p.S = S;
+  p.D = D;
+  p.causal = causal ? 1 : 0;
+  p.n_pairs = (S + ROWS - 1) / ROWS;
+  const long long items = BH * p.n_pairs;
+  if (items > INT_MAX) return RA_ERR_SHAPE;
+  p.n_items = static_cast<int>(items);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  constexpr int smem = Layout<HD>::ALLOC;
+  const int slot = HD == 128 ? 0 : 1;
+  if (!di->fwd_attr[slot]) {
+    const cudaError_t e = cudaFuncSetAttribute(fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(fwd smem)");
+    di->fwd_attr[slot] = true;
+  }
+  const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
+  fwd_kernel<HD><<<grid, NUM_THREADS, smem, stream>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+int fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int S, int Dh, int D,
+            int causal, float scale, cudaStream_t stream) {
+  using namespace ra::f32;
+  const long long rows = static_cast<long long>(B) * H * S;
+  const long long blocks = (rows + WARPS - 1) / WARPS;
+  if (blocks > INT_MAX) return RA_ERR_SHAPE;
+  const int vpl = (Dh + 31) / 32;
+#define RA_F32_CASE(N)                                                                                         \
+  case N:                                                                                                      \
+    fwd_f32_kernel<N><<<static_cast<int>(blocks), WARPS * 32, 0, stream>>>(q, k, v, o, lse, rows, S, Dh, D,  \
+                                                                           causal, scale);                   \
+    break;
+  switch (vpl) {
+    RA_F32_CASE(1) RA_F32_CASE(2) RA_F32_CASE(3) RA_F32_CASE(4) RA_F32_CASE(5) RA_F32_CASE(6) RA_F32_CASE(7)
+    RA_F32_CASE(8)
+    default:
+      return RA_ERR_SHAPE;
+  }
+#undef RA_F32_CASE
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int ring_attn_version(void) { return RA_VERSION; }
+
+int ring_attn_last_cuda_error(const char** site) {
+  if (site) *site = g_last_cuda_site;
+  return g_last_cuda_code;
+}
+
+const char* ring_attn_strerror(int code) {
+  switch (code) {
+    case RA_OK: return "ok";
+    case RA_ERR_ARG: return "invalid argument (null pointer, non-positive size or unknown dtype)";
+    case RA_ERR_SHAPE: return "unsupported shape (S % D != 0, D > S, unsupported head dim or size overflow)";
+    case RA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case RA_ERR_WORKSPACE: return "workspace missing or too small";
+    case RA_ERR_CUDA: return "CUDA runtime/driver call failed";
+    case RA_ERR_TIMEOUT: return "a kernel gave up on a bounded internal wait";
+    case RA_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    default: return "unknown status code";
+  }
+}
+
+int ring_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int Dh,
+                     int D, int causal, ra_dtype dtype, float scale, ra_stream stream) {
+  if (!q || !k || !v || !o || !lse) return RA_ERR_ARG;
+  if (dtype != RA_BF16 && dtype != RA_F32) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  const float sc = (scale > 0.f && std::isfinite(scale)) ? scale : 1.0f / std::sqrt(static_cast<float>(Dh));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == RA_F32) {
+    if (Dh > 256) return RA_ERR_SHAPE;
+    int dst = RA_OK;
+    if (!dev_info(&dst)) return dst;
+    return fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+                   static_cast<float*>(o), lse, B, H, S, Dh, D, causal, sc, s);
+  }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RA_ERR_ALIGN;
+  if (Dh == 128) return fwd_bf16<128>(q, k, v, o, lse, B, H, S, D, causal, sc, s);
+  if (Dh == 64) return fwd_bf16<64>(q, k, v, o, lse, B, H, S, D, causal, sc, s);
+  return RA_ERR_SHAPE;
+}
+
+int ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int Dh, int D,
+                  int causal, ra_stream stream) {
+  return ring_attn_fwd_ex(q, k, v, o, lse, B, H, S, Dh, D, causal, RA_BF16, 0.f, stream);
+}
+
+int ring_attn_merge_ex(const float* o_parts, const float* lse_parts, int P, void* o, float* lse, int B, int H, int S,
+                       int Dh, ra_dtype out_dtype, ra_stream stream) {
+  if (!o_parts || !lse_parts || !o || !lse) return RA_ERR_ARG;
+  if (P <= 0 || B <= 0 || H <= 0 || S <= 0 || Dh <= 0) return RA_ERR_ARG;
+  if (out_dtype != RA_BF16 && out_dtype != RA_F32) return RA_ERR_ARG;
+  if (Dh % 4 != 0 || Dh > 256) return RA_ERR_SHAPE;
+  if (!aligned16(o_parts) || !aligned16(o)) return RA_ERR_ALIGN;
+  const long long rows = static_cast<long long>(B) * H * S;
+  if (static_cast<double>(rows) * P * Dh > 9.0e18 / 4) return RA_ERR_SHAPE;
+  int st = RA_OK;
+  if (!dev_info(&st)) return st;
+  const long long blocks = (rows + ra::merge::WARPS - 1) / ra::merge::WARPS;
+  if (blocks > INT_MAX) return RA_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (out_dtype == RA_BF16)
+    ra::merge::merge_kernel<__nv_bfloat16><<<static_cast<int>(blocks), ra::merge::WARPS * 32, 0, s>>>(
+        o_parts, lse_parts, P, static_cast<__nv_bfloat16*>(o), lse, rows, Dh);
+  else
+    ra::merge::merge_kernel<float><<<static_cast<int>(blocks), ra::merge::WARPS * 32, 0, s>>>(
+        o_parts, lse_parts, P, static_cast<float*>(o), lse, rows, Dh);
+  return launch_status();
+}
+
+int ring_attn_merge(const float* o_parts, const float* lse_parts, int P, void* o, float* lse, int B, int H, int S,
+                    int Dh, ra_stream stream) {
+  return ring_attn_merge_ex(o_parts, lse_parts, P, o, lse, B, H, S, Dh, RA_BF16, stream);
+}
+
+int ring_attn_ring_order(int D, int r, int causal, int* blocks, int max_blocks) {
+  if (D <= 0 || r < 0 || r >= D || !blocks) return -RA_ERR_ARG;
+  int n = 0;
+  for (int t = 0; t < D; ++t) {
+    const int j = ((r - t) % D + D) % D;
+    if (causal && j > r) continue;
+    if (n >= max_blocks) return -RA_ERR_ARG;
+    blocks[n++] = j;
+  }
+  return n;
+}
+
+int ring_attn_visit_tiles(int S, int D, int causal, int q0, int tile_rows, int* tiles, int max_tiles) {
+  if (S <= 0 || D <= 0 || D > S || S % D != 0 || q0 < 0 || q0 >= S || tile_rows <= 0 || !tiles)
+    return -RA_ERR_ARG;
+  ra::RingTiles it;
+  it.init(S, D, causal, q0, tile_rows, ra::fwd::BN);
+  int n = 0;
+  for (int kt = it.next(); kt >= 0; kt = it.next()) {
+    if (n >= max_tiles) return -RA_ERR_ARG;
+    tiles[n++] = kt;
+  }
+  return n;
+}
+
+int ring_attn_device_status(ra_stream stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ra::g_status, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  if (v != 0) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(ra::g_status, &z, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"
+
+// --- backward entry points (kernel in bwd_sm100.cuh) ---
+extern "C" {
+size_t ring_attn_bwd_workspace_size(int B, int H, int S, int Dh) {
+  if (B <= 0 || H <= 0 || S <= 0 || Dh <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * S;
+  const size_t a = (rows * Dh * 4 + 255) & ~size_t(255);
+  const size_t b = (rows * 4 + 255) & ~size_t(255);
+  return a + b;
+}
+
+int ring_attn_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
+                  void*, int, int, int, int, int, int, void*, size_t, ra_stream) {
+  return RA_ERR_SHAPE;
+}
+}

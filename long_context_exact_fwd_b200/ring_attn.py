@@ -1,0 +1,196 @@
+"""ctypes binding of libringattn.so (include/ring_attn.h): argument marshalling only.
+
+Every step of the forward, backward and merge runs in the library's CUDA kernels; this
+module only checks tensor properties, allocates outputs with torch (device memory
+plumbing) and passes raw pointers plus the current CUDA stream.  There is no fallback:
+importing this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libringattn.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m long_context_exact_fwd_b200.build` "
+        "(there is no CPU fallback)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+RA_OK, RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_ALIGN, RA_ERR_WORKSPACE, RA_ERR_CUDA, RA_ERR_TIMEOUT, RA_ERR_DEVICE = range(8)
+RA_BF16, RA_F32 = 0, 1
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_ip = ctypes.POINTER(ctypes.c_int)
+
+
+def _sig(name, restype, *argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+_fwd = _sig("ring_attn_fwd", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
+_fwd_ex = _sig("ring_attn_fwd_ex", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp)
+_bwd_ws = _sig("ring_attn_bwd_workspace_size", _sz, _i, _i, _i, _i)
+_bwd = _sig("ring_attn_bwd", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
+_merge_ex = _sig("ring_attn_merge_ex", _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp)
+_ring_order = _sig("ring_attn_ring_order", _i, _i, _i, _i, _ip, _i)
+_visit_tiles = _sig("ring_attn_visit_tiles", _i, _i, _i, _i, _i, _i, _ip, _i)
+_device_status = _sig("ring_attn_device_status", _i, _vp)
+_strerror = _sig("ring_attn_strerror", ctypes.c_char_p, _i)
+_version = _sig("ring_attn_version", _i)
+_last_cuda = _sig("ring_attn_last_cuda_error", _i, ctypes.POINTER(ctypes.c_char_p))
+
+
+class RingAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = f"{where}: status {code} ({strerror(code)})"
+        if code == RA_ERR_CUDA:
+            err, site = last_cuda_error()
+            msg += f"; last CUDA failure {err} in {site}"
+        super().__init__(msg)
+
+
+def last_cuda_error() -> Tuple[int, str]:
+    site = ctypes.c_char_p()
+    code = _last_cuda(ctypes.byref(site))
+    return int(code), (site.value or b"").decode()
+
+
+def strerror(code: int) -> str:
+    return _strerror(code).decode()
+
+
+def version() -> int:
+    return _version()
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def _check(code: int, where: str) -> None:
+    if code != RA_OK:
+        raise RingAttnError(code, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, D: int, causal: bool = True,
+        scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+        lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Ring-attention forward.  q, k, v: [B, H, S, Dh] bf16 (or float32) CUDA tensors.
+    Returns (o [B, H, S, Dh] in the input dtype, lse [B, H, S] float32)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, S, Dh]")
+    B, H, S, Dh = q.shape
+    dt = q.dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise ValueError("inputs must be bfloat16 or float32")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, dt, q.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _need(out, "out", dt, q.shape)
+    _need(lse, "lse", torch.float32, (B, H, S))
+    code = _fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, S, Dh, D,
+                   1 if causal else 0, RA_BF16 if dt == torch.bfloat16 else RA_F32,
+                   float(scale) if scale else 0.0, _stream(stream))
+    _check(code, "ring_attn_fwd")
+    return out, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, S: int, Dh: int) -> int:
+    return int(_bwd_ws(B, H, S, Dh))
+
+
+def bwd(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=None,
+        workspace: Optional[torch.Tensor] = None, stream=None):
+    """Ring-attention backward (bf16).  Returns (dq, dk, dv), each [B, H, S, Dh] bf16."""
+    B, H, S, Dh = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, name, torch.bfloat16, q.shape)
+    _need(lse, "lse", torch.float32, (B, H, S))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, torch.bfloat16, q.shape)
+    need = bwd_workspace_bytes(B, H, S, Dh)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    code = _bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, Dh, D, 1 if causal else 0,
+                workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "ring_attn_bwd")
+    return dq, dk, dv
+
+
+def merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.bfloat16,
+          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
+    """LSE merge of P partials: o_parts [P, B, H, S, Dh] f32, lse_parts [P, B, H, S] f32."""
+    P, B, H, S, Dh = o_parts.shape
+    _need(o_parts, "o_parts", torch.float32)
+    _need(lse_parts, "lse_parts", torch.float32, (P, B, H, S))
+    if out is None:
+        out = torch.empty((B, H, S, Dh), dtype=out_dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=o_parts.device)
+    _need(out, "out", out_dtype, (B, H, S, Dh))
+    _need(lse, "lse", torch.float32, (B, H, S))
+    code = _merge_ex(o_parts.data_ptr(), lse_parts.data_ptr(), P, out.data_ptr(), lse.data_ptr(), B, H, S, Dh,
+                     RA_BF16 if out_dtype == torch.bfloat16 else RA_F32, _stream(stream))
+    _check(code, "ring_attn_merge")
+    return out, lse
+
+
+def ring_order(D: int, r: int, causal: bool) -> List[int]:
+    """Host-side ring schedule of the library (blocks visited by position r, in order)."""
+    buf = (ctypes.c_int * max(D, 1))()
+    n = _ring_order(D, r, 1 if causal else 0, buf, D)
+    if n < 0:
+        raise RingAttnError(-n, "ring_attn_ring_order")
+    return list(buf[:n])
+
+
+def visit_tiles(S: int, D: int, causal: bool, q0: int, rows: int) -> List[int]:
+    """Host-side copy of the forward kernel's key-tile visit order for one query tile."""
+    cap = S // 128 + 2
+    buf = (ctypes.c_int * cap)()
+    n = _visit_tiles(S, D, 1 if causal else 0, q0, rows, buf, cap)
+    if n < 0:
+        raise RingAttnError(-n, "ring_attn_visit_tiles")
+    return list(buf[:n])
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device status word."""
+    return int(_device_status(_stream(stream)))
+
+
+# raw entry points (for tests of the C ABI itself)
+raw = _lib

@@ -1,0 +1,118 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared symbol,
+validates arguments before touching the device, and its host-side ring schedule matches
+the oracle's ring order and the pages' worked example."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"RA_API\s+[\w\s\*]+?\b(ring_attn_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for required in ("ring_attn_fwd", "ring_attn_bwd", "ring_attn_merge"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib_path):
+    lib = ctypes.CDLL(lib_path)
+    missing = [n for n in _declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+@pytest.fixture(scope="module")
+def ra(lib_path):
+    from long_context_exact_fwd_b200 import ring_attn
+    return ring_attn
+
+
+def test_version_and_strerror(ra):
+    assert ra.version() >= 100
+    for code in range(8):
+        assert isinstance(ra.strerror(code), str) and ra.strerror(code)
+    assert "unknown" in ra.strerror(999)
+
+
+def test_argument_errors_are_reported_before_any_device_work(ra):
+    f = ra.raw.ring_attn_fwd_ex
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    args = lambda **kw: [P(kw.get("q", 16)), P(16), P(16), P(16), P(16), kw.get("B", 1), 2, kw.get("S", 256),
+                         kw.get("Dh", 128), kw.get("D", 4), 1, kw.get("dtype", 0), ctypes.c_float(0.0), P(0)]
+    assert f(*args(q=0)) == ra.RA_ERR_ARG                 # null pointer
+    assert f(*args(B=0)) == ra.RA_ERR_ARG                 # non-positive size
+    assert f(*args(dtype=7)) == ra.RA_ERR_ARG             # unknown dtype
+    assert f(*args(S=250, D=4)) == ra.RA_ERR_SHAPE        # uneven ring split
+    assert f(*args(S=4, D=8)) == ra.RA_ERR_SHAPE          # more blocks than tokens
+    assert f(*args(q=18)) == ra.RA_ERR_ALIGN              # misaligned TMA source
+    assert f(*args(Dh=96)) in (ra.RA_ERR_SHAPE,)          # no bf16 kernel for Dh=96
+    # valid arguments on a machine without a usable sm_100 device: reported, not crashed
+    import torch
+    if not torch.cuda.is_available():
+        assert f(*args()) in (ra.RA_ERR_CUDA, ra.RA_ERR_DEVICE)
+
+
+def test_merge_and_bwd_argument_errors(ra):
+    m = ra.raw.ring_attn_merge_ex
+    P = ctypes.c_void_p
+    assert m(P(0), P(16), 2, P(16), P(16), 1, 1, 8, 128, 0, P(0)) == ra.RA_ERR_ARG
+    assert m(P(16), P(16), 0, P(16), P(16), 1, 1, 8, 128, 0, P(0)) == ra.RA_ERR_ARG
+    assert m(P(16), P(16), 2, P(16), P(16), 1, 1, 8, 126, 0, P(0)) == ra.RA_ERR_SHAPE
+    assert ra.bwd_workspace_bytes(1, 2, 256, 128) >= 1 * 2 * 256 * 128 * 4 + 1 * 2 * 256 * 4
+    assert ra.bwd_workspace_bytes(0, 2, 256, 128) == 0
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_library_ring_order_matches_oracle(ra, causal):
+    for D in (1, 2, 3, 4, 7, 8, 16):
+        for r in range(D):
+            assert ra.ring_order(D, r, causal) == oracle.ring_order(D, r, causal)
+
+
+def test_library_ring_order_reproduces_the_pages_worked_example(ra):
+    rows = [tuple(int(x) for x in ln.split())
+            for ln in open(os.path.join(ROOT, "tests", "golden", "ring_walkthrough_d4.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    for dev, rnd, blk in rows:
+        assert ra.ring_order(4, dev, False)[rnd - 1] == blk
+
+
+def _expected_tiles(S, D, causal, q0, rows, KT=128):
+    """Independent restatement: ring order of the tile's block, each block's tiles
+    (first key inside the block) ascending, tiles beyond the last query row dropped."""
+    c = S // D
+    q_last = min(q0 + rows, S) - 1
+    out = []
+    for j in oracle.ring_order(D, q0 // c, False):
+        for kt in range(-(-j * c // KT), -(-(j + 1) * c // KT)):
+            if causal and kt * KT > q_last:
+                continue
+            out.append(kt)
+    return out
+
+
+@pytest.mark.parametrize("S,D", [(256, 1), (1024, 4), (8192, 8), (1000, 8), (384, 3), (1536, 6), (130, 2),
+                                 (4096, 16), (257, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_visit_tiles_schedule_and_coverage(ra, S, D, causal):
+    n_tiles = -(-S // 128)
+    for q0 in range(0, S, 256):
+        got = ra.visit_tiles(S, D, causal, q0, 256)
+        assert got == _expected_tiles(S, D, causal, q0, 256)
+        # every key tile holding a key visible to some row of the query tile, exactly once
+        last = min(q0 + 256, S) - 1
+        need = [kt for kt in range(n_tiles) if not causal or kt * 128 <= last]
+        assert sorted(got) == need
