@@ -91,9 +91,10 @@ RA_API int ring_attn_fwd_ex(const void* q, const void* k, const void* v, void* o
                      int Dh, int D, int causal, ra_dtype dtype, float scale, ra_stream stream);
 
 /*
- * ring_attn_bwd_workspace_size -- bytes of device workspace ring_attn_bwd needs:
- * a float32 dQ accumulator [B][H][S][Dh] and a float32 row statistic [B][H][S] (Delta),
- * each 256-byte aligned.  Returns 0 for invalid sizes.
+ * ring_attn_bwd_workspace_size -- bytes of device workspace ring_attn_bwd needs: a float32
+ * dQ accumulator [B][H][S][Dh] and two float32 row statistics (Delta = rowsum(dO * O) and
+ * lse * log2(e)) of [B][H][S_pad] with S_pad = S rounded up to 128, each region 256-byte
+ * aligned.  Returns 0 for invalid sizes.
  */
 RA_API size_t ring_attn_bwd_workspace_size(int B, int H, int S, int Dh);
 
@@ -151,6 +152,21 @@ RA_API int ring_attn_ring_order(int D, int r, int causal, int* blocks, int max_b
  * tiles[0..n) and returns n, or -RA_ERR_ARG.
  */
 RA_API int ring_attn_visit_tiles(int S, int D, int causal, int q0, int tile_rows, int* tiles, int max_tiles);
+
+/*
+ * ring_attn_bwd_visit_tiles -- host only.  The backward's query-tile visit order for the
+ * key tile starting at key k0: key/value block j = k0 / (S / D) is at ring position
+ * (j + t) mod D at step t, so the tile visits, for t = 0..D-1, the `tile_rows`-row query
+ * tiles whose first row lies in block (j + t) mod D, ascending, dropping (causal) tiles that
+ * end before k0.  Writes query tile indices to tiles[0..n) and returns n, or -RA_ERR_ARG.
+ */
+RA_API int ring_attn_bwd_visit_tiles(int S, int D, int causal, int k0, int tile_rows, int* tiles, int max_tiles);
+
+/*
+ * ring_attn_launch_count -- number of CUDA kernels this library has launched since it was
+ * loaded (all host threads and devices); for accounting in benchmarks.
+ */
+RA_API unsigned long long ring_attn_launch_count(void);
 
 /*
  * ring_attn_device_status -- synchronises `stream`, returns the device status word

@@ -1,1 +1,513 @@
+// Backward ring-attention kernels for sm_100a.
+//
+// The pages ("精读笔记 · Ring Attention with Blockwise Transformers for Near-Infinite
+// Context", §4.2 and the BPT background of §2.2) state that training runs through the same
+// blockwise ring structure but give no formulas; this is the analytic softmax gradient with
+// P recomputed from the forward's log-sum-exp:
+//   P = exp(scale q k^T - lse), dV = P^T dO, dP = dO V^T, Delta = rowsum(dO * O),
+//   dS = P * (dP - Delta), dQ = scale dS K, dK = scale dS^T Q.
+//
+// Three kernels:
+//   bwd_pre     Delta (fp32), lse * log2(e) (fp32), both padded per head to a multiple of
+//               128 rows, and a zeroed fp32 dQ accumulator (HBM-bound).
+//   bwd_kernel  key/value-stationary: one CTA per (head, 128-key tile) at a time, visiting
+//               the query tiles that can see the key tile in ring order (ring step t brings
+//               the key/value block j to the position of query block (j + t) mod D, step 0
+//               being its own block); dK, dV accumulate in TMEM, dQ is added atomically to
+//               the fp32 accumulator.
+//   bwd_convert dQ = scale * accumulator -> bf16 (HBM-bound).
+//
+// bwd_kernel CTA (384 threads):
+//   warpgroup 0  thread = key row: P^T, dS^T (bf16) into TMEM and dS into shared memory;
+//                final dK, dV epilogue.
+//   warpgroup 1  thread = query row: reads the two dQ halves from TMEM, red.add to global.
+//   warp 8       TMA producer: K, V once per item; Q, dO, lse2, Delta per query tile (2 stages).
+//   warp 9       TMEM allocator + tcgen05.mma issuer.
+// TMEM (512 columns): [0,128) S^T, P^T (bf16) in [0,64), dQ[:, 0:64] in [64,128);
+//   [128,256) dP^T, dS^T (bf16) in [128,192), dQ[:, 64:128] in [192,256);
+//   [256,384) dV; [384,512) dK.
+// MMAs per query tile (M = 128, K = 128 each): S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
+//   dK += dS^T Q, dQ(two N = 64 halves) = dS K.
 #pragma once
+#include "ra_schedule.h"
+#include "ra_sm100.cuh"
+
+namespace ra {
+namespace bwd {
+
+constexpr int BM = 128;   // keys per CTA tile (TMEM lanes of S^T, dP^T, dV, dK)
+constexpr int BQ = 128;   // queries per query tile
+constexpr int HD = 128;   // head dimension of this kernel
+constexpr int NSTAGE = 2;
+constexpr int NUM_THREADS = 384;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
+// Registers: launched at 168.  Warpgroup 2 lowers to 88 (frees 128 x 80); warpgroup 0
+// raises to 248 (takes 128 x 80); warpgroup 1 keeps 168.
+constexpr uint32_t REGS_LAUNCH = 168, REGS_WG0 = 248, REGS_OTHER = 88;
+static_assert(REGS_WG0 - REGS_LAUNCH <= REGS_LAUNCH - REGS_OTHER, "register split exceeds the pool");
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_S = 0, COL_DQ0 = 64, COL_DP = 128, COL_DS = 128, COL_DQ1 = 192, COL_DV = 256, COL_DK = 384;
+
+struct Layout {
+  static constexpr int SUB_BYTES = 128 * 128;          // 128 rows x 128 B (64 bf16)
+  static constexpr int TILE_BYTES = 2 * SUB_BYTES;     // 128 rows x 128 bf16
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + TILE_BYTES;
+  static constexpr int DS_OFF = V_OFF + TILE_BYTES;    // dS, MN-major: two 64-query halves
+  static constexpr int STAGE_OFF = DS_OFF + TILE_BYTES;
+  static constexpr int STAGE_Q = 0, STAGE_DO = TILE_BYTES, STAGE_LSE = 2 * TILE_BYTES,
+                       STAGE_DELTA = STAGE_LSE + BQ * 4, STAGE_BYTES = STAGE_DELTA + BQ * 4;
+  static constexpr int BAR_OFF = STAGE_OFF + NSTAGE * STAGE_BYTES;
+  static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_QD_FULL = 2, B_QD_EMPTY = B_QD_FULL + NSTAGE,
+                       B_S_FULL = B_QD_EMPTY + NSTAGE, B_DP_FULL = B_S_FULL + 1, B_P_READY = B_DP_FULL + 1,
+                       B_DS_READY = B_P_READY + 1, B_DQ_FULL = B_DS_READY + 1, B_DQ_FREE = B_DQ_FULL + 1,
+                       B_ACC_FULL = B_DQ_FREE + 1, B_DRAIN = B_ACC_FULL + 1, NUM_BARS = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+};
+static_assert(Layout::BYTES <= 232448, "shared memory");
+
+struct Params {
+  int BH, S, S_pad, D, causal;
+  int n_kt;              // key tiles per head
+  int n_items;           // BH * n_kt
+  float scale_log2;      // scale * log2(e)
+  float scale;
+  const float* lse2;     // [BH][S_pad] lse * log2(e), +inf in padding
+  const float* delta;    // [BH][S_pad]
+  float* dq_acc;         // [BH][S][HD] fp32
+  __nv_bfloat16* dk;     // [BH][S][HD]
+  __nv_bfloat16* dv;
+};
+
+using RingQTiles = ::ra::RingQTiles;
+
+// Work item w -> (bh, key tile).  Causal: the first key tiles see the most query tiles.
+__device__ __forceinline__ void item_coords(int w, const Params& p, int& bh, int& kt) {
+  const int rank = w / p.BH;
+  bh = w - rank * p.BH;
+  kt = rank;
+}
+
+__device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
+  if (++stage == NSTAGE) {
+    stage = 0;
+    phase ^= 1u;
+  }
+}
+
+// ------------------------------------------------------------------ producer
+__device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                         const CUtensorMap* tm_do, const Params& p, uint32_t sbase, volatile int* abort_flag) {
+  using L = Layout;
+  auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
+  int stage = 0;
+  uint32_t phase = 0, kv_phase = 0;
+  uint32_t issued = 0, issued_parity = 0, kv_issued = 0, kv_parity = 0;
+  bool ok = true;
+  for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+    int bh, kt;
+    item_coords(w, p, bh, kt);
+    if (!mbar_wait(bar(L::B_KV_EMPTY), kv_phase ^ 1u, abort_flag)) { ok = false; break; }
+    mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * L::TILE_BYTES);
+    for (int sb = 0; sb < 2; ++sb) {
+      tma_load_3d(tm_k, sbase + L::K_OFF + sb * L::SUB_BYTES, bar(L::B_KV_FULL), sb * 64, kt * BM, bh);
+      tma_load_3d(tm_v, sbase + L::V_OFF + sb * L::SUB_BYTES, bar(L::B_KV_FULL), sb * 64, kt * BM, bh);
+    }
+    kv_issued = 1;
+    kv_parity = kv_phase;
+    kv_phase ^= 1u;
+    RingQTiles it;
+    it.init(p.S, p.D, p.causal, kt * BM, BQ);
+    for (int qt = it.next(); qt >= 0; qt = it.next()) {
+      if (!mbar_wait(bar(L::B_QD_EMPTY + stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+      const uint32_t full = bar(L::B_QD_FULL + stage);
+      const uint32_t st = sbase + L::STAGE_OFF + stage * L::STAGE_BYTES;
+      mbar_arrive_expect_tx(full, 2 * L::TILE_BYTES + 2 * BQ * 4);
+      for (int sb = 0; sb < 2; ++sb) {
+        tma_load_3d(tm_q, st + L::STAGE_Q + sb * L::SUB_BYTES, full, sb * 64, qt * BQ, bh);
+        tma_load_3d(tm_do, st + L::STAGE_DO + sb * L::SUB_BYTES, full, sb * 64, qt * BQ, bh);
+      }
+      const size_t row0 = static_cast<size_t>(bh) * p.S_pad + static_cast<size_t>(qt) * BQ;
+      bulk_load(st + L::STAGE_LSE, p.lse2 + row0, BQ * 4, full);
+      bulk_load(st + L::STAGE_DELTA, p.delta + row0, BQ * 4, full);
+      issued |= 1u << stage;
+      issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+      advance(stage, phase);
+    }
+  }
+  if (!ok) {
+    for (int s = 0; s < NSTAGE; ++s)
+      if (issued & (1u << s)) drain_wait(bar(L::B_QD_FULL + s), (issued_parity >> s) & 1u);
+    if (kv_issued) drain_wait(bar(L::B_KV_FULL), kv_parity);
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, bool first_zero) {
+  // D[128 x 128] = A[128 x 128] * B[128 x 128]^T, both K-major 128-B swizzled (two 64-col halves)
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * Layout::SUB_BYTES + (kk & 3) * 32;
+    umma_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), IDESC,
+            (first_zero && kk == 0) ? 0u : 1u);
+  }
+}
+
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
+  // D[128 x 128] (+)= A[128 x 128] (TMEM, bf16) * B[128 x 128] (smem, MN-major: rows = K)
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, HD, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < BQ / 16; ++kk)
+    umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC,
+            (accumulate || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ void mma_dq_half(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_half_smem) {
+  // dQ[:, h] [128 q x 64] = dS [128 q x 128 k] (MN-major: q contiguous, two 64-q halves)
+  //                        * K[:, h] [128 k x 64] (MN-major: rows = K)
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, 64, 1, 1);
+#pragma unroll
+  for (int kk = 0; kk < BM / 16; ++kk)
+    umma_ss(d_tmem, sdesc_sw128(ds_smem + kk * 2048, Layout::SUB_BYTES, 1024),
+            sdesc_sw128(k_half_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC, kk > 0 ? 1u : 0u);
+}
+
+__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+  using L = Layout;
+  auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
+  int stage = 0;
+  uint32_t phase = 0, kv_phase = 0, p_phase = 0, ds_phase = 0, dqf_phase = 0;
+  bool ok = true;
+  bool dq_pending = false;   // a dQ readout of the previous query tile is outstanding
+  for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+    int bh, kt;
+    item_coords(w, p, bh, kt);
+    if (!mbar_wait(bar(L::B_KV_FULL), kv_phase, abort_flag)) { ok = false; break; }
+    kv_phase ^= 1u;
+    tc_fence_after();
+    RingQTiles it;
+    it.init(p.S, p.D, p.causal, kt * BM, BQ);
+    int n = 0;
+    for (int qt = it.next(); qt >= 0; qt = it.next(), ++n) {
+      const int s = stage;
+      const uint32_t st = sbase + L::STAGE_OFF + s * L::STAGE_BYTES;
+      if (!mbar_wait(bar(L::B_QD_FULL + s), phase, abort_flag)) { ok = false; break; }
+      advance(stage, phase);
+      if (dq_pending) {  // S^T and dP^T overwrite the columns the dQ readout is reading
+        if (!mbar_wait(bar(L::B_DQ_FREE), dqf_phase, abort_flag)) { ok = false; break; }
+        dqf_phase ^= 1u;
+      }
+      tc_fence_after();
+      mma_kmajor(tmem + COL_S, sbase + L::K_OFF, st + L::STAGE_Q, true);     // S^T = K Q^T
+      tc_commit(bar(L::B_S_FULL));
+      mma_kmajor(tmem + COL_DP, sbase + L::V_OFF, st + L::STAGE_DO, true);   // dP^T = V dO^T
+      tc_commit(bar(L::B_DP_FULL));
+      if (!mbar_wait(bar(L::B_P_READY), p_phase, abort_flag)) { ok = false; break; }
+      p_phase ^= 1u;
+      tc_fence_after();
+      mma_tmem_a(tmem + COL_DV, tmem + COL_S, st + L::STAGE_DO, n > 0);     // dV += P^T dO
+      if (!mbar_wait(bar(L::B_DS_READY), ds_phase, abort_flag)) { ok = false; break; }
+      ds_phase ^= 1u;
+      tc_fence_after();
+      mma_tmem_a(tmem + COL_DK, tmem + COL_DS, st + L::STAGE_Q, n > 0);     // dK += dS^T Q
+      tc_commit(bar(L::B_QD_EMPTY + s));                                       // Q, dO, lse2, Delta free
+      mma_dq_half(tmem + COL_DQ0, sbase + L::DS_OFF, sbase + L::K_OFF);
+      mma_dq_half(tmem + COL_DQ1, sbase + L::DS_OFF, sbase + L::K_OFF + L::SUB_BYTES);
+      tc_commit(bar(L::B_DQ_FULL));
+      dq_pending = true;
+    }
+    if (!ok) break;
+    tc_commit(bar(L::B_ACC_FULL));   // dV, dK final once everything issued so far completes
+    tc_commit(bar(L::B_KV_EMPTY));   // K, V (read by the last dQ MMAs) free then too
+  }
+  tc_commit(bar(L::B_DRAIN));
+  drain_wait(bar(L::B_DRAIN), 0);
+}
+
+// ------------------------------------------------------------------ warpgroup 0: P^T, dS^T, epilogue
+__device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+  using L = Layout;
+  auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
+  const int lane = threadIdx.x & 31;
+  const int quarter = (threadIdx.x >> 5) & 3;
+  const int row = quarter * 32 + lane;   // key row within the tile
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  const float sl2 = p.scale_log2;
+  int stage = 0;
+  uint32_t phase = 0, s_phase = 0, dp_phase = 0, acc_phase = 0;
+  // dS row of this thread in the MN-major shared tile: half h (queries 64h..64h+63), 16-B
+  // chunk c of the 128-B row goes to chunk c ^ (row & 7) (128-byte swizzle).
+  uint8_t* ds_row = smem + L::DS_OFF + row * 128;
+  const int sw = row & 7;
+
+  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+    int bh, kt;
+    item_coords(w, p, bh, kt);
+    const int k_row = kt * BM + row;
+    RingQTiles it;
+    it.init(p.S, p.D, p.causal, kt * BM, BQ);
+    for (int qt = it.next(); qt >= 0; qt = it.next()) {
+      const float* lse2 = reinterpret_cast<const float*>(smem + L::STAGE_OFF + stage * L::STAGE_BYTES + L::STAGE_LSE);
+      const float* dlt = reinterpret_cast<const float*>(smem + L::STAGE_OFF + stage * L::STAGE_BYTES + L::STAGE_DELTA);
+      // lse2 / Delta arrive by bulk copy on the stage's full barrier: observe it directly
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QD_FULL + stage), phase, abort_flag))) return;
+      advance(stage, phase);
+      const int q0 = qt * BQ;
+      // visible queries of this key row: [lo, hi) in tile coordinates
+      const int lo = p.causal ? k_row - q0 : 0;
+      const int hi = (k_row < p.S) ? p.S - q0 : 0;
+      const bool masked = (lo > 0) || (hi < BQ);
+
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_S_FULL), s_phase, abort_flag))) return;
+      s_phase ^= 1u;
+      tc_fence_after();
+      float pv[BQ];
+      {
+        uint32_t r[BQ];
+#pragma unroll
+        for (int c = 0; c < BQ / 32; ++c)
+          tmem_ld32(lane_base + COL_S + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < BQ; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
+          pv[c + 0] = ex2_approx(fmaf(__uint_as_float(r[c + 0]), sl2, -l4.x));
+          pv[c + 1] = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, -l4.y));
+          pv[c + 2] = ex2_approx(fmaf(__uint_as_float(r[c + 2]), sl2, -l4.z));
+          pv[c + 3] = ex2_approx(fmaf(__uint_as_float(r[c + 3]), sl2, -l4.w));
+        }
+      }
+      if (masked) {
+#pragma unroll
+        for (int c = 0; c < BQ; ++c)
+          if (c < lo || c >= hi) pv[c] = 0.f;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {   // P^T (bf16) -> TMEM columns [0, 64)
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[64 * h + 2 * c], pv[64 * h + 2 * c + 1]);
+        tmem_st32(lane_base + COL_S + 32 * h, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_P_READY));
+
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DP_FULL), dp_phase, abort_flag))) return;
+      dp_phase ^= 1u;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < BQ / 32; ++ch) {   // 32 queries per chunk
+        uint32_t d[32];
+        tmem_ld32(lane_base + COL_DP + 32 * ch, d);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 dl = *reinterpret_cast<const float2*>(dlt + 32 * ch + c);
+          const float a = pv[32 * ch + c] * (__uint_as_float(d[c]) - dl.x);
+          const float b = pv[32 * ch + c + 1] * (__uint_as_float(d[c + 1]) - dl.y);
+          pk[c >> 1] = pack_bf16x2(a, b);
+        }
+        tmem_st16(lane_base + COL_DS + 16 * ch, pk);
+        // shared dS: queries 32ch..32ch+31 = half ch/2, 16-B chunks 4(ch&1) .. +3
+        uint8_t* half = ds_row + (ch >> 1) * L::SUB_BYTES;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int chunk = ((ch & 1) * 4 + j) ^ sw;
+          *reinterpret_cast<uint4*>(half + chunk * 16) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();   // generic-proxy dS stores -> visible to the tensor core
+      tc_fence_before();
+      mbar_arrive(bar(L::B_DS_READY));
+    }
+    // epilogue: dV, dK (scaled) for this key tile
+    if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC_FULL), acc_phase, abort_flag))) return;
+    acc_phase ^= 1u;
+    tc_fence_after();
+    const bool row_ok = k_row < p.S;
+    const size_t off = (static_cast<size_t>(bh) * p.S + k_row) * HD;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t col = which ? COL_DK : COL_DV;
+      const float mul = which ? p.scale : 1.f;
+      __nv_bfloat16* dst_row = (which ? p.dk : p.dv) + off;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + col + 32 * c, r);
+        tmem_ld_wait();
+        uint32_t w16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w16[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ warpgroup 1: dQ readout
+__device__ void query_rows_wg(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+  using L = Layout;
+  auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
+  const int lane = threadIdx.x & 31;
+  const int quarter = (threadIdx.x >> 5) & 3;
+  const int row = quarter * 32 + lane;   // query row within the tile
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  uint32_t phase = 0;
+  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+    int bh, kt;
+    item_coords(w, p, bh, kt);
+    RingQTiles it;
+    it.init(p.S, p.D, p.causal, kt * BM, BQ);
+    for (int qt = it.next(); qt >= 0; qt = it.next()) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQ_FULL), phase, abort_flag))) return;
+      phase ^= 1u;
+      tc_fence_after();
+      const int q_row = qt * BQ + row;
+      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.S + q_row) * HD;
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(lane_base + ((c < 2) ? COL_DQ0 + 32 * c : COL_DQ1 + 32 * (c - 2)),
+                  *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_DQ_FREE));   // both halves are in registers: hand the columns back
+      if (q_row < p.S) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          atomicAdd(reinterpret_cast<float4*>(dst + 4 * i),
+                    make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ main kernel
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
+  using L = Layout;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  const int warp = threadIdx.x >> 5;
+  if (sbase & 1023u) {   // the 128-byte swizzle needs 1024-byte aligned tiles
+    if (threadIdx.x == 0) record_status(RA_ERR_CUDA);
+    return;              // uniform: every thread sees the same base
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NUM_BARS; ++i) {
+      const bool many = (i == L::B_P_READY || i == L::B_DS_READY || i == L::B_DQ_FREE);
+      mbar_init(sbase + L::BAR_OFF + 8u * i, many ? 128 : 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == WARP_TMA && (threadIdx.x & 31) == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= 8) {
+    regs_lower<REGS_OTHER>();
+    if (warp == WARP_TMA) {
+      if ((threadIdx.x & 31) == 0) producer(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
+      __syncwarp();
+    } else if (warp == WARP_MMA) {
+      if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, abort_flag);
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    regs_raise<REGS_WG0>();
+    key_rows_wg(p, smem, sbase, tmem, abort_flag);
+  } else {
+    query_rows_wg(p, sbase, tmem, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ preprocess / convert
+constexpr int PRE_WARPS = 8;
+
+// One warp per padded row: Delta = sum_d dO * O, lse2 = lse * log2(e) (+inf and 0 in the
+// padding rows), and the row of the fp32 dQ accumulator cleared.
+__global__ void __launch_bounds__(PRE_WARPS * 32)
+    bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                   const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
+                   float* __restrict__ dq_acc, int BH, int S, int S_pad) {
+  const int lane = threadIdx.x & 31;
+  const long long prow = static_cast<long long>(blockIdx.x) * PRE_WARPS + (threadIdx.x >> 5);
+  if (prow >= static_cast<long long>(BH) * S_pad) return;
+  const long long bh = prow / S_pad;
+  const int s = static_cast<int>(prow - bh * S_pad);
+  if (s >= S) {
+    if (lane == 0) {
+      delta[prow] = 0.f;
+      lse2[prow] = INFINITY;
+    }
+    return;
+  }
+  const long long row = bh * S + s;
+  // HD = 128 bf16 per row: 8 bytes (4 values) per lane
+  const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + row * HD) + lane);
+  const uint2 b = __ldg(reinterpret_cast<const uint2*>(dO + row * HD) + lane);
+  const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+  const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float2 fa = __bfloat1622float2(a2[i]), fb = __bfloat1622float2(b2[i]);
+    acc = fmaf(fa.x, fb.x, acc);
+    acc = fmaf(fa.y, fb.y, acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  reinterpret_cast<float4*>(dq_acc + row * HD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane == 0) {
+    delta[prow] = acc;
+    lse2[prow] = lse[row] * 1.4426950408889634f;
+  }
+}
+
+// dQ = scale * accumulator -> bf16, 8 elements per thread.
+__global__ void __launch_bounds__(256)
+    bwd_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, long long n8, float scale) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i);
+  const float4 b = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i + 1);
+  reinterpret_cast<uint4*>(dq)[i] = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                                               pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+}
+
+}  // namespace bwd
+}  // namespace ra

@@ -56,4 +56,40 @@ struct RingTiles {
   }
 };
 
+// The backward's view of the same ring: key/value block j sits at ring position
+// (j + t) mod D at step t, so a key tile [k0, k0 + 128) visits, for t = 0..D-1, the query
+// tiles of `qt_size` rows whose first row lies in block (j + t) mod D, ascending; under the
+// causal mask, query tiles whose last row precedes k0 see none of its keys and are dropped.
+struct RingQTiles {
+  int D, c, qt_size, t, j, qt, qt_end, qt_min, n_qt;
+
+  RA_HD void init(int S, int D_, int causal, int k0, int qt_size_) {
+    D = D_;
+    c = S / D_;
+    qt_size = qt_size_;
+    j = k0 / c;
+    t = 0;
+    n_qt = RingTiles::cdiv(S, qt_size);
+    qt_min = causal ? k0 / qt_size : 0;   // tile i ends at row qt_size * (i + 1) - 1
+    set_block();
+  }
+
+  RA_HD void set_block() {
+    const int p = (j + t) % D;
+    const int a = RingTiles::cdiv(static_cast<long long>(p) * c, qt_size);
+    const int b = RingTiles::cdiv(static_cast<long long>(p + 1) * c, qt_size);
+    qt = a > qt_min ? a : qt_min;
+    qt_end = b < n_qt ? b : n_qt;
+  }
+
+  // Next query tile index in visit order, or -1.
+  RA_HD int next() {
+    while (t < D) {
+      if (qt < qt_end) return qt++;
+      if (++t < D) set_block();
+    }
+    return -1;
+  }
+};
+
 }  // namespace ra

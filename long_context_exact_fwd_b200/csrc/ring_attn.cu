@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -29,6 +30,9 @@ int cuda_fail(int code, const char* site) {
 }
 
 constexpr int RA_VERSION = 100;
+
+// Kernels this library has launched (all threads, all devices) since load.
+std::atomic<unsigned long long> g_launches{0};
 constexpr int MAX_DEVICES = 64;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -117,6 +121,7 @@ int check_shape(int B, int H, int S, int Dh, int D) {
 }
 
 int launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : cuda_fail(static_cast<int>(e), "kernel launch");
 }
@@ -176,6 +181,86 @@ int fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse
       return RA_ERR_SHAPE;
   }
 #undef RA_F32_CASE
+  return launch_status();
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdWorkspace {
+  size_t dq_bytes, row_bytes, total;
+};
+
+BwdWorkspace bwd_workspace(long long BH, int S, int Dh) {
+  const long long S_pad = (static_cast<long long>(S) + 127) / 128 * 128;
+  BwdWorkspace w;
+  w.dq_bytes = align256(static_cast<size_t>(BH) * S * Dh * 4);
+  w.row_bytes = align256(static_cast<size_t>(BH) * S_pad * 4);
+  w.total = w.dq_bytes + 2 * w.row_bytes;
+  return w;
+}
+
+int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+             void* dk, void* dv, int B, int H, int S, int D, int causal, float scale, void* workspace,
+             cudaStream_t stream) {
+  namespace rb = ra::bwd;
+  int st = RA_OK;
+  DevInfo* di = dev_info(&st);
+  if (!di) return st;
+  const long long BH = static_cast<long long>(B) * H;
+  const BwdWorkspace ws = bwd_workspace(BH, S, rb::HD);
+  const int S_pad = (S + 127) / 128 * 128;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.dq_bytes);
+  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.dq_bytes + ws.row_bytes);
+
+  // 1. Delta, lse * log2(e), cleared dQ accumulator
+  const long long prow = BH * S_pad;
+  const long long pre_blocks = (prow + rb::PRE_WARPS - 1) / rb::PRE_WARPS;
+  if (pre_blocks > INT_MAX) return RA_ERR_SHAPE;
+  rb::bwd_pre_kernel<<<static_cast<int>(pre_blocks), rb::PRE_WARPS * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, delta, lse2, dq_acc,
+      static_cast<int>(BH), S, S_pad);
+  if ((st = launch_status()) != RA_OK) return st;
+
+  // 2. key/value-stationary main kernel
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_map(&mq, q, BH, S, rb::HD, rb::BQ)) != RA_OK) return st;
+  if ((st = make_map(&mk, k, BH, S, rb::HD, rb::BM)) != RA_OK) return st;
+  if ((st = make_map(&mv, v, BH, S, rb::HD, rb::BM)) != RA_OK) return st;
+  if ((st = make_map(&mdo, dO, BH, S, rb::HD, rb::BQ)) != RA_OK) return st;
+  rb::Params p;
+  p.BH = static_cast<int>(BH);
+  p.S = S;
+  p.S_pad = S_pad;
+  p.D = D;
+  p.causal = causal ? 1 : 0;
+  p.n_kt = (S + rb::BM - 1) / rb::BM;
+  const long long items = BH * p.n_kt;
+  if (items > INT_MAX) return RA_ERR_SHAPE;
+  p.n_items = static_cast<int>(items);
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  constexpr int smem = rb::Layout::BYTES;
+  if (!di->bwd_attr) {
+    const cudaError_t e = cudaFuncSetAttribute(rb::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(bwd smem)");
+    di->bwd_attr = true;
+  }
+  const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
+  rb::bwd_kernel<<<grid, rb::NUM_THREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  if ((st = launch_status()) != RA_OK) return st;
+
+  // 3. dQ = scale * accumulator -> bf16
+  const long long n8 = BH * S * rb::HD / 8;
+  const long long cblocks = (n8 + 255) / 256;
+  if (cblocks > INT_MAX) return RA_ERR_SHAPE;
+  rb::bwd_convert_kernel<<<static_cast<int>(cblocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8,
+                                                                       scale);
   return launch_status();
 }
 
@@ -296,18 +381,45 @@ int ring_attn_device_status(ra_stream stream) {
 
 }  // extern "C"
 
-// --- backward entry points (kernel in bwd_sm100.cuh) ---
+
 extern "C" {
+
 size_t ring_attn_bwd_workspace_size(int B, int H, int S, int Dh) {
   if (B <= 0 || H <= 0 || S <= 0 || Dh <= 0) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * S;
-  const size_t a = (rows * Dh * 4 + 255) & ~size_t(255);
-  const size_t b = (rows * 4 + 255) & ~size_t(255);
-  return a + b;
+  return bwd_workspace(static_cast<long long>(B) * H, S, Dh).total;
 }
 
-int ring_attn_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
-                  void*, int, int, int, int, int, int, void*, size_t, ra_stream) {
-  return RA_ERR_SHAPE;
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D, int causal, void* workspace,
+                  size_t workspace_bytes, ra_stream stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  if (Dh != ra::bwd::HD) return RA_ERR_SHAPE;
+  for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return RA_ERR_ALIGN;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < ring_attn_bwd_workspace_size(B, H, S, Dh))
+    return RA_ERR_WORKSPACE;
+  const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
+  return bwd_bf16(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, workspace,
+                  static_cast<cudaStream_t>(stream));
 }
+
+int ring_attn_bwd_visit_tiles(int S, int D, int causal, int k0, int tile_rows, int* tiles, int max_tiles) {
+  if (S <= 0 || D <= 0 || D > S || S % D != 0 || k0 < 0 || k0 >= S || tile_rows <= 0 || !tiles)
+    return -RA_ERR_ARG;
+  ra::RingQTiles it;
+  it.init(S, D, causal, k0, tile_rows);
+  int n = 0;
+  for (int qt = it.next(); qt >= 0; qt = it.next()) {
+    if (n >= max_tiles) return -RA_ERR_ARG;
+    tiles[n++] = qt;
+  }
+  return n;
 }
+
+unsigned long long ring_attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -45,6 +45,8 @@ _device_status = _sig("ring_attn_device_status", _i, _vp)
 _strerror = _sig("ring_attn_strerror", ctypes.c_char_p, _i)
 _version = _sig("ring_attn_version", _i)
 _last_cuda = _sig("ring_attn_last_cuda_error", _i, ctypes.POINTER(ctypes.c_char_p))
+_bwd_visit_tiles = _sig("ring_attn_bwd_visit_tiles", _i, _i, _i, _i, _i, _i, _ip, _i)
+_launch_count = _sig("ring_attn_launch_count", ctypes.c_ulonglong)
 
 
 class RingAttnError(RuntimeError):
@@ -185,6 +187,21 @@ def visit_tiles(S: int, D: int, causal: bool, q0: int, rows: int) -> List[int]:
     if n < 0:
         raise RingAttnError(-n, "ring_attn_visit_tiles")
     return list(buf[:n])
+
+
+def bwd_visit_tiles(S: int, D: int, causal: bool, k0: int, rows: int = 128) -> List[int]:
+    """Host-side copy of the backward kernel's query-tile visit order for one key tile."""
+    cap = S // max(rows, 1) + 2
+    buf = (ctypes.c_int * cap)()
+    n = _bwd_visit_tiles(S, D, 1 if causal else 0, k0, rows, buf, cap)
+    if n < 0:
+        raise RingAttnError(-n, "ring_attn_bwd_visit_tiles")
+    return list(buf[:n])
+
+
+def launch_count() -> int:
+    """Kernels launched by the library since it was loaded."""
+    return int(_launch_count())
 
 
 def device_status(stream=None) -> int:

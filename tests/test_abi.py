@@ -116,3 +116,39 @@ def test_visit_tiles_schedule_and_coverage(ra, S, D, causal):
         last = min(q0 + 256, S) - 1
         need = [kt for kt in range(n_tiles) if not causal or kt * 128 <= last]
         assert sorted(got) == need
+
+
+def _expected_q_tiles(S, D, causal, k0, rows=128):
+    """Independent restatement for the backward: block j of the key tile travels the ring,
+    visiting query blocks j, j+1, ... (mod D); each block's query tiles (first row inside
+    the block) ascending; under the causal mask tiles ending before k0 are dropped."""
+    c = S // D
+    j = k0 // c
+    out = []
+    for t in range(D):
+        p = (j + t) % D
+        for qt in range(-(-p * c // rows), -(-(p + 1) * c // rows)):
+            if causal and (qt + 1) * rows - 1 < k0:
+                continue
+            out.append(qt)
+    return out
+
+
+@pytest.mark.parametrize("S,D", [(256, 1), (1024, 4), (8192, 8), (1000, 8), (384, 3), (130, 2), (16384, 8)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_visit_tiles_schedule_and_coverage(ra, S, D, causal):
+    n_qt = -(-S // 128)
+    for k0 in range(0, S, 128):
+        got = ra.bwd_visit_tiles(S, D, causal, k0)
+        assert got == _expected_q_tiles(S, D, causal, k0)
+        need = [qt for qt in range(n_qt) if not causal or (qt + 1) * 128 - 1 >= k0]
+        assert sorted(got) == need
+
+
+def test_bwd_ring_order_is_the_forward_ring_seen_from_the_key_side():
+    """At ring step t query block r meets key block (r - t) mod D (forward view) exactly
+    when key block j meets query block (j + t) mod D (backward view)."""
+    D = 8
+    for r in range(D):
+        for t, j in enumerate(oracle.ring_order(D, r, False)):
+            assert (j + t) % D == r
