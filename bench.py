@@ -1,0 +1,389 @@
+"""Benchmark of the exact ring-attention hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over the workload: ring_attn_fwd (forward,
+online softmax over the ring, LSE) then ring_attn_bwd (Delta preprocess, key/value-
+stationary backward, dQ convert) for the default 16K-token forward+backward workload;
+forward-only workloads run ring_attn_fwd alone.  Inputs are seeded synthetic tensors
+already resident in HBM.  The metric is causal-adjusted TFLOP/s (forward 4*B*H*S^2*Dh/2,
+backward 2.5x forward).  Multi-GPU (torchrun): every rank runs its own seeded replica of
+the workload (weak scaling, no collective on the data path); time is the max over ranks.
+
+--impl reference times the float64 CPU oracle on bounded samples of the same workload
+(rank 0 only) and prints the same line shape with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_exact_fwd_b200.workloads import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "ring-attn fwd/bwd TFLOP/s & % of BF16 tensor peak, S=8K–128K, 1 B200"
+DEFAULT_WORKLOAD = "s16k_fwd_bwd"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CSRC = os.path.join(ROOT, "long_context_exact_fwd_b200", "csrc")
+
+
+# ------------------------------------------------------------------------------- helpers
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _csrc_digest() -> str:
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("csrc_sha") == _csrc_digest():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def _cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        pw = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower().startswith("active")})
+        top = max(sm) if sm else 0
+        loaded = [s for s in sm if s >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------------------- reference arm
+def oracle_sample(w: Workload, inp, sample_rows: int):
+    """Time the float64 oracle on a bounded sample of the workload; returns
+    (causal-adjusted flops of the sample, seconds, description)."""
+    import oracle
+    import numpy as np
+    q = inp["q"][0, 0].double().numpy()
+    k = inp["k"][0, 0].double().numpy()
+    v = inp["v"][0, 0].double().numpy()
+    if w.backward:
+        n = min(w.S, sample_rows)   # causal prefix: a complete causal problem of its own
+        do = inp["do"][0, 0].double().numpy()
+        t0 = time.perf_counter()
+        oracle.attn_fwd(q[:n], k[:n], v[:n], w.causal)
+        oracle.attn_bwd(q[:n], k[:n], v[:n], do[:n], w.causal)
+        dt = time.perf_counter() - t0
+        f = 4.0 * n * n * w.Dh * (0.5 if w.causal else 1.0) * 3.5
+        return f, dt, f"head (0,0), first {n} tokens (causal prefix), forward + backward"
+    rng = np.random.default_rng(w.seed + 2000)
+    rows = np.sort(rng.choice(w.S, size=min(sample_rows, w.S), replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, w.causal, rows=rows)
+    dt = time.perf_counter() - t0
+    vis = (rows + 1).sum() if w.causal else rows.size * w.S
+    f = 4.0 * w.Dh * float(vis)
+    return f, dt, f"head (0,0), {rows.size} random query rows, forward"
+
+
+def run_reference(args, w: Workload):
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    inp = make_inputs(w)
+    n = args.sample_rows or (4096 if w.backward else 1024)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, n)
+    flops = secs = 0.0
+    desc = ""
+    for _ in range(args.steps):
+        f, dt, desc = oracle_sample(w, inp, n)
+        flops += f
+        secs += dt
+    value = flops / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, args),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": f"{desc}, per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w: Workload, args):
+    ws_bytes = 2 * w.B * w.H * w.S * w.Dh * (9 if w.backward else 4)
+    return {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "Dh": w.Dh, "D": w.D, "causal": w.causal,
+            "pass": "fwd+bwd" if w.backward else "fwd", "flops_per_step": w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0),
+            "l2": ("working set %.0f MiB > %d MiB L2, not flushed" % (ws_bytes / 2 ** 20, L2_BYTES >> 20))
+            if ws_bytes > 3 * L2_BYTES else "L2 flushed between steps (256 MiB write)",
+            "seeds": f"workload seed {w.seed} (+1000*rank)"}
+
+
+# ------------------------------------------------------------------------------- our arm
+def run_ours(args, w: Workload):
+    import torch
+    import torch.distributed as dist
+    from long_context_exact_fwd_b200 import ring_attn as ra
+
+    ws, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    host = make_inputs(wr)
+    names = ("q", "k", "v", "do") if w.backward else ("q", "k", "v")
+    x = {n: host[n].to(dev) for n in names}
+    o = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    if w.backward:
+        dq, dk, dv = (torch.empty_like(x["q"]) for _ in range(3))
+        wsb = torch.empty(ra.bwd_workspace_bytes(w.B, w.H, w.S, w.Dh), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush_needed = "flushed" in _config(w, args)["l2"]
+    flush_buf = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev) if flush_needed else None
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ra.fwd(x["q"], x["k"], x["v"], w.D, w.causal, out=o, lse=lse, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        if w.backward:
+            ra.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], w.D, w.causal, dq, dk, dv, workspace=wsb, stream=stream)
+            if evs:
+                evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ra.device_status(stream) != 0:
+        raise RuntimeError("device status not clean after warm-up")
+
+    n_ev = 3 if w.backward else 2
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = ra.launch_count()
+    with ClockSampler(uuid) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            if flush_buf is not None:
+                flush_buf.fill_(float(i))
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall
+    launches = ra.launch_count() - launches0
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    st = ra.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed region")
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if w.backward else [0.0] * args.steps
+    step_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, gradients (or O) back out
+    pinned = {n: host[n].pin_memory() for n in names}
+    outs = ("dq", "dk", "dv") if w.backward else ("o", "lse")
+    h_out = {n: torch.empty((w.B, w.H, w.S, w.Dh) if n != "lse" else (w.B, w.H, w.S),
+                            dtype=torch.float32 if n == "lse" else w.torch_dtype).pin_memory() for n in outs}
+    dev_out = {"dq": dq, "dk": dk, "dv": dv} if w.backward else {"o": o, "lse": lse}
+    h2d = sum(t_.numel() * t_.element_size() for t_ in pinned.values())
+    d2h = sum(t_.numel() * t_.element_size() for t_ in h_out.values())
+
+    def e2e_step():
+        for n in names:
+            x[n].copy_(pinned[n], non_blocking=True)
+        step()
+        for n in outs:
+            h_out[n].copy_(dev_out[n], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(te.item())
+
+    flops_step = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
+    value = ws * flops_step * args.steps / (max_total_ms * 1e-3) / 1e12
+    e2e_value = ws * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12
+
+    if rank == 0:
+        peaks, src = _peaks()
+        long_region = t_wall > 2.0
+        peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+        f_ms, b_ms = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+        kernels = {"ring_attn_fwd": {"ms": f_ms, "tflops": w.fwd_flops() / (f_ms * 1e-3) / 1e12}}
+        if w.backward:
+            kernels["ring_attn_bwd"] = {"ms": b_ms, "tflops": w.bwd_flops() / (b_ms * 1e-3) / 1e12}
+        dom = "ring_attn_bwd" if (w.backward and b_ms >= f_ms) else "ring_attn_fwd"
+        dom_kernel = "bwd_kernel" if dom == "ring_attn_bwd" else "fwd_kernel"
+        achieved = kernels[dom]["tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": _traffic(dom_kernel, w.name), "kernel": dom_kernel,
+                "peak_source": f"{src} {'sustained' if long_region else 'burst'} bf16 dense "
+                               f"(MEASURED_PEAKS.json)" if src == "measured" else "fallback",
+                "timing": ("CUDA events around the %s call on its stream over the timed region" % dom)
+                + (" (includes its Delta preprocess and dQ convert kernels)" if dom == "ring_attn_bwd" else "")}
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            n = args.sample_rows or (w.S if w.backward else 2048)
+            f, dt, desc = oracle_sample(w, host, n)
+            cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
+                   "sample": desc + f" ({dt:.1f} s)"}
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {**_config(w, args), "parallelism": f"replicas x{ws} (no data-path collective)"},
+                "pct_of_bf16_peak": 100.0 * value / ws / peak,
+                "roofline": roof, "kernels": kernels, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches, "clocks": clocks.summary()}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[n for n in WORKLOADS if n != "tiny_fp32"])
+    ap.add_argument("--sample-rows", type=int, default=0, help="oracle sample size (rows / causal prefix)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)   # the timing rules ask for at least 3 warm-up steps
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
