@@ -118,6 +118,32 @@ RA_API int ring_attn_bwd(const void* q, const void* k, const void* v, const void
                   size_t workspace_bytes, ra_stream stream);
 
 /*
+ * ring_attn_bwd_noalloc -- ring_attn_bwd for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for callers that may not call
+ * cudaMalloc (or any allocator) on their path -- for example code embedded in a host
+ * framework that owns every device allocation, or latency-critical code that cannot afford
+ * cudaMalloc's implicit synchronisation -- and so cannot supply ring_attn_bwd's workspace.
+ *   Arguments are those of ring_attn_bwd without the workspace.  The fp32 dQ accumulator and
+ *   the per-row statistics live instead in one static device array of the library of
+ *   ring_attn_bwd_noalloc_max_bytes() bytes (96 MiB), reserved on every device that loads the
+ *   library until the process exits.  A problem whose ring_attn_bwd_workspace_size exceeds that
+ *   size is rejected with RA_ERR_WORKSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture.  No call allocates
+ *   or frees memory.
+ *   Every call on a device shares the one array, which keeps the previous call's contents; each
+ *   call clears the accumulator it needs on the stream before use.  Calls whose execution
+ *   overlaps on the GPU (different streams, or concurrent host threads) race on the array and
+ *   give wrong gradients: serialise them.
+ */
+RA_API int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                 const void* dO, void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D,
+                                 int causal, ra_stream stream);
+
+/* ring_attn_bwd_noalloc_max_bytes -- size of ring_attn_bwd_noalloc's static scratch array. */
+RA_API size_t ring_attn_bwd_noalloc_max_bytes(void);
+
+/*
  * ring_attn_merge -- combine P normalised partial outputs through their log-sum-exp
  * (page "精读笔记 ...", §3.1: blocks may be combined in any order when their statistics are
  * combined with rescaling; page "RingAttention large-context attention", 架构与算法: the

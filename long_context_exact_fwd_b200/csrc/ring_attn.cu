@@ -423,3 +423,60 @@ int ring_attn_bwd_visit_tiles(int S, int D, int causal, int k0, int tile_rows, i
 unsigned long long ring_attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// --- backward without caller-provided workspace -------------------------------------------
+// Scratch for ring_attn_bwd_noalloc: the fp32 dQ accumulator and the two per-row statistics
+// live in this file-scope device array instead of a caller buffer.  Every device that loads
+// the library holds RA_NOALLOC_SCRATCH_BYTES for it until the process exits.
+namespace {
+
+constexpr size_t RA_NOALLOC_SCRATCH_BYTES = 96ull << 20;   // 96 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device, looked up once per device
+// (host code may not use the array's name as a device pointer).
+int scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return cuda_fail(static_cast<int>(e), "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(static_cast<int>(e), "cudaGetSymbolAddress(noalloc scratch)");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ring_attn_bwd_noalloc_max_bytes(void) { return RA_NOALLOC_SCRATCH_BYTES; }
+
+int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D,
+                          int causal, ra_stream stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  if (Dh != ra::bwd::HD) return RA_ERR_SHAPE;
+  for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return RA_ERR_ALIGN;
+  if (ring_attn_bwd_workspace_size(B, H, S, Dh) > RA_NOALLOC_SCRATCH_BYTES) return RA_ERR_WORKSPACE;
+  int dst = RA_OK;
+  if (!dev_info(&dst)) return dst;
+  void* scratch = nullptr;
+  if ((st = scratch_address(&scratch)) != RA_OK) return st;
+  const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
+  return bwd_bf16(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, scratch,
+                  static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -47,6 +47,8 @@ _version = _sig("ring_attn_version", _i)
 _last_cuda = _sig("ring_attn_last_cuda_error", _i, ctypes.POINTER(ctypes.c_char_p))
 _bwd_visit_tiles = _sig("ring_attn_bwd_visit_tiles", _i, _i, _i, _i, _i, _i, _ip, _i)
 _launch_count = _sig("ring_attn_launch_count", ctypes.c_ulonglong)
+_bwd_noalloc = _sig("ring_attn_bwd_noalloc", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
+_noalloc_max = _sig("ring_attn_bwd_noalloc_max_bytes", _sz)
 
 
 class RingAttnError(RuntimeError):
@@ -150,6 +152,30 @@ def bwd(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=N
                 workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "ring_attn_bwd")
     return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=None, stream=None):
+    """Backward through ring_attn_bwd_noalloc: no workspace argument; the library's static
+    device scratch (bwd_noalloc_max_bytes()) holds the dQ accumulator.  Calls that overlap
+    on the GPU race on that scratch."""
+    B, H, S, Dh = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, name, torch.bfloat16, q.shape)
+    _need(lse, "lse", torch.float32, (B, H, S))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, torch.bfloat16, q.shape)
+    code = _bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, Dh, D, 1 if causal else 0,
+                        _stream(stream))
+    _check(code, "ring_attn_bwd_noalloc")
+    return dq, dk, dv
+
+
+def bwd_noalloc_max_bytes() -> int:
+    return int(_noalloc_max())
 
 
 def merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.bfloat16,
