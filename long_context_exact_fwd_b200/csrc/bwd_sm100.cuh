@@ -13,14 +13,16 @@
 //   bwd_kernel  key/value-stationary: one CTA per (head, 128-key tile) at a time, visiting
 //               the query tiles that can see the key tile in ring order (ring step t brings
 //               the key/value block j to the position of query block (j + t) mod D, step 0
-//               being its own block); dK, dV accumulate in TMEM, dQ is added atomically to
-//               the fp32 accumulator.
+//               being its own block); dK, dV accumulate in TMEM, dQ partials are added to
+//               the fp32 accumulator by TMA bulk reduce-add.
 //   bwd_convert dQ = scale * accumulator -> bf16 (HBM-bound).
 //
 // bwd_kernel CTA (384 threads):
 //   warpgroup 0  thread = key row: P^T, dS^T (bf16) into TMEM and dS into shared memory;
 //                final dK, dV epilogue.
-//   warpgroup 1  thread = query row: reads the two dQ halves from TMEM, red.add to global.
+//   warpgroup 1  thread = query row: reads dQ from TMEM, stages it (fp32, 128-B swizzled
+//                32-column boxes) in the dS buffer once the dQ MMAs have consumed dS, and one
+//                thread issues TMA reduce-adds into the fp32 accumulator.
 //   warp 8       TMA producer: K, V once per item; Q, dO, lse2, Delta per query tile (2 stages).
 //   warp 9       TMEM allocator + tcgen05.mma issuer.
 // TMEM (512 columns): [0,128) S^T, P^T (bf16) in [0,64), dQ[:, 0:64] in [64,128);
@@ -31,6 +33,7 @@
 #pragma once
 #include "ra_schedule.h"
 #include "ra_sm100.cuh"
+#include "ra_work.cuh"
 
 namespace ra {
 namespace bwd {
@@ -61,8 +64,10 @@ struct Layout {
   static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_QD_FULL = 2, B_QD_EMPTY = B_QD_FULL + NSTAGE,
                        B_S_FULL = B_QD_EMPTY + NSTAGE, B_DP_FULL = B_S_FULL + 1, B_P_READY = B_DP_FULL + 1,
                        B_DS_READY = B_P_READY + 1, B_DQ_FULL = B_DS_READY + 1, B_DQ_FREE = B_DQ_FULL + 1,
-                       B_ACC_FULL = B_DQ_FREE + 1, B_DRAIN = B_ACC_FULL + 1, NUM_BARS = B_DRAIN + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+                       B_ACC_FULL = B_DQ_FREE + 1, B_DS_FREE = B_ACC_FULL + 1, B_DRAIN = B_DS_FREE + 1,
+                       B_WQ_FULL = B_DRAIN + 1, B_WQ_EMPTY = B_WQ_FULL + 2, NUM_BARS = B_WQ_EMPTY + 2;
+  static constexpr uint32_t WQ_CONSUMERS = 1 + 8;   // MMA thread + one arrival per warp of warpgroups 0, 1
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, item ring[2]
   static constexpr int BYTES = MISC_OFF + 16;
 };
 static_assert(Layout::BYTES <= 232448, "shared memory");
@@ -71,6 +76,8 @@ struct Params {
   int BH, S, S_pad, D, causal;
   int n_kt;              // key tiles per head
   int n_items;           // BH * n_kt
+  int hgroup;            // heads whose items are interleaved (L2 reuse of Q, dO)
+  int work_slot;         // this launch's work counter
   float scale_log2;      // scale * log2(e)
   float scale;
   const float* lse2;     // [BH][S_pad] lse * log2(e), +inf in padding
@@ -82,11 +89,16 @@ struct Params {
 
 using RingQTiles = ::ra::RingQTiles;
 
-// Work item w -> (bh, key tile).  Causal: the first key tiles see the most query tiles.
+// Work item w -> (bh, key tile).  Heads are taken in groups of p.hgroup whose Q/dO fit in
+// L2 together; inside a group items go key tile by key tile (causal: the first key tiles
+// see the most query tiles, so the longest items come first).
 __device__ __forceinline__ void item_coords(int w, const Params& p, int& bh, int& kt) {
-  const int rank = w / p.BH;
-  bh = w - rank * p.BH;
-  kt = rank;
+  const int per_group = p.hgroup * p.n_kt;
+  const int g = w / per_group;
+  const int gsize = min(p.hgroup, p.BH - g * p.hgroup);
+  const int idx = w - g * per_group;
+  kt = idx / gsize;
+  bh = g * p.hgroup + (idx - kt * gsize);
 }
 
 __device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
@@ -98,14 +110,20 @@ __device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
 
 // ------------------------------------------------------------------ producer
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                         const CUtensorMap* tm_do, const Params& p, uint32_t sbase, volatile int* abort_flag) {
+                         const CUtensorMap* tm_do, const Params& p, uint32_t sbase, volatile int* wq,
+                         volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
   uint32_t issued = 0, issued_parity = 0, kv_issued = 0, kv_parity = 0;
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  int w = work_fetch(p.work_slot);
+  for (;;) {
+    if (!ring.push(w, abort_flag)) { ok = false; break; }
+    if (w >= p.n_items) break;
+    const int w_next = work_fetch(p.work_slot);
     int bh, kt;
     item_coords(w, p, bh, kt);
     if (!mbar_wait(bar(L::B_KV_EMPTY), kv_phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -135,7 +153,10 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
       issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
       advance(stage, phase);
     }
+    if (!ok) break;
+    w = w_next;
   }
+  work_done(p.work_slot);
   if (!ok) {
     for (int s = 0; s < NSTAGE; ++s)
       if (issued & (1u << s)) drain_wait(bar(L::B_QD_FULL + s), (issued_parity >> s) & 1u);
@@ -174,14 +195,18 @@ __device__ __forceinline__ void mma_dq_half(uint32_t d_tmem, uint32_t ds_smem, u
             sdesc_sw128(k_half_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC, kk > 0 ? 1u : 0u);
 }
 
-__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0, p_phase = 0, ds_phase = 0, dqf_phase = 0;
   bool ok = true;
   bool dq_pending = false;   // a dQ readout of the previous query tile is outstanding
-  for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (;;) {
+    int w;
+    if (!ring.pop(w, abort_flag)) { ok = false; break; }
+    if (w >= p.n_items) break;
     int bh, kt;
     item_coords(w, p, bh, kt);
     if (!mbar_wait(bar(L::B_KV_FULL), kv_phase, abort_flag)) { ok = false; break; }
@@ -227,7 +252,8 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
 }
 
 // ------------------------------------------------------------------ warpgroup 0: P^T, dS^T, epilogue
-__device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem, volatile int* wq,
+                            volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   const int lane = threadIdx.x & 31;
@@ -236,13 +262,17 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
   const float sl2 = p.scale_log2;
   int stage = 0;
-  uint32_t phase = 0, s_phase = 0, dp_phase = 0, acc_phase = 0;
+  uint32_t phase = 0, s_phase = 0, dp_phase = 0, acc_phase = 0, dsf_phase = 0;
   // dS row of this thread in the MN-major shared tile: half h (queries 64h..64h+63), 16-B
   // chunk c of the 128-B row goes to chunk c ^ (row & 7) (128-byte swizzle).
   uint8_t* ds_row = smem + L::DS_OFF + row * 128;
   const int sw = row & 7;
 
-  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (;;) {
+    int w;
+    if (!ring.pop_warp(w, abort_flag)) return;
+    if (w >= p.n_items) break;
     int bh, kt;
     item_coords(w, p, bh, kt);
     const int k_row = kt * BM + row;
@@ -297,6 +327,10 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
 
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DP_FULL), dp_phase, abort_flag))) return;
       dp_phase ^= 1u;
+      // the dS buffer doubles as dQ staging of the previous query tile: wait until its
+      // reduce-adds have read it
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DS_FREE), dsf_phase ^ 1u, abort_flag))) return;
+      dsf_phase ^= 1u;
       tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < BQ / 32; ++ch) {   // 32 queries per chunk
@@ -356,53 +390,84 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
 }
 
 // ------------------------------------------------------------------ warpgroup 1: dQ readout
-__device__ void query_rows_wg(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                              volatile int* wq, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   const int lane = threadIdx.x & 31;
   const int quarter = (threadIdx.x >> 5) & 3;
   const int row = quarter * 32 + lane;   // query row within the tile
+  const bool leader = (threadIdx.x & 127) == 0;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  uint8_t* stage_row = smem + L::DS_OFF + row * 128;
+  const int sw = row & 7;
   uint32_t phase = 0;
-  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+  bool ok = true;
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (;;) {
+    int w = 0;
+    // warpgroup-uniform outcome (the named barriers below need all four warps)
+    ok = named_bar_and(1, 128, ring.pop_warp(w, abort_flag));
+    if (!ok || w >= p.n_items) break;
     int bh, kt;
     item_coords(w, p, bh, kt);
     RingQTiles it;
     it.init(p.S, p.D, p.causal, kt * BM, BQ);
     for (int qt = it.next(); qt >= 0; qt = it.next()) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQ_FULL), phase, abort_flag))) return;
+      // every thread of the warpgroup reaches this barrier (the wait is bounded), so the
+      // named barriers below never wait for a thread that gave up
+      ok = named_bar_and(1, 128, mbar_wait(bar(L::B_DQ_FULL), phase, abort_flag));
+      if (!ok) break;
       phase ^= 1u;
       tc_fence_after();
-      const int q_row = qt * BQ + row;
-      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.S + q_row) * HD;
-      uint32_t r[128];
+      uint32_t r[HD];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         tmem_ld32(lane_base + ((c < 2) ? COL_DQ0 + 32 * c : COL_DQ1 + 32 * (c - 2)),
                   *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::B_DQ_FREE));   // both halves are in registers: hand the columns back
-      if (q_row < p.S) {
+      mbar_arrive(bar(L::B_DQ_FREE));   // dQ is in registers: hand the TMEM columns back
+      // dQ row -> four 32-column fp32 boxes (128 B per row, 128-B swizzle), two per round
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          atomicAdd(reinterpret_cast<float4*>(dst + 4 * i),
-                    make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+      for (int round = 0; round < 2; ++round) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const int c0 = 32 * (2 * round + b);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(stage_row + b * L::SUB_BYTES + ((j ^ sw) << 4)) =
+                make_uint4(r[c0 + 4 * j], r[c0 + 4 * j + 1], r[c0 + 4 * j + 2], r[c0 + 4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            tma_reduce_add_3d(tm_dq, sbase + L::DS_OFF + b * L::SUB_BYTES, 32 * (2 * round + b), qt * BQ, bh);
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+        named_bar_sync(1, 128);   // staging may be overwritten
       }
+      if (leader) mbar_arrive(bar(L::B_DS_FREE));
     }
+    if (!ok) break;
   }
+  if (leader) bulk_wait_all();   // reduce-adds complete before the CTA exits
 }
 
 // ------------------------------------------------------------------ main kernel
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const __grid_constant__ CUtensorMap tm_dq, const Params p) {
   using L = Layout;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  volatile int* wq = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
   const int warp = threadIdx.x >> 5;
   if (sbase & 1023u) {   // the 128-byte swizzle needs 1024-byte aligned tiles
     if (threadIdx.x == 0) record_status(RA_ERR_CUDA);
@@ -411,7 +476,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       const bool many = (i == L::B_P_READY || i == L::B_DS_READY || i == L::B_DQ_FREE);
-      mbar_init(sbase + L::BAR_OFF + 8u * i, many ? 128 : 1);
+      const bool wq_empty = (i >= L::B_WQ_EMPTY && i < L::B_WQ_EMPTY + 2);
+      mbar_init(sbase + L::BAR_OFF + 8u * i, many ? 128 : (wq_empty ? L::WQ_CONSUMERS : 1));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -425,6 +491,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -434,17 +501,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp >= 8) {
     regs_lower<REGS_OTHER>();
     if (warp == WARP_TMA) {
-      if ((threadIdx.x & 31) == 0) producer(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
+      if ((threadIdx.x & 31) == 0) producer(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, wq, abort_flag);
       __syncwarp();
     } else if (warp == WARP_MMA) {
-      if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, abort_flag);
+      if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, wq, abort_flag);
       __syncwarp();
     }
   } else if (warp < 4) {
     regs_raise<REGS_WG0>();
-    key_rows_wg(p, smem, sbase, tmem, abort_flag);
+    key_rows_wg(p, smem, sbase, tmem, wq, abort_flag);
   } else {
-    query_rows_wg(p, sbase, tmem, abort_flag);
+    query_rows_wg(p, &tm_dq, smem, sbase, tmem, wq, abort_flag);
   }
 
   tc_fence_before();

@@ -7,7 +7,7 @@
 // with block compute -- here the on-chip analogue: the K/V tiles of the next steps are in
 // flight through TMA while the tensor cores work on the current one).
 //
-// CTA = one work item at a time (persistent grid, static round robin over items):
+// CTA = one work item at a time (persistent grid; items taken from a global counter):
 //   item = (b*H + h, pair of query tiles Q0 = rows [256i, 256i+128), Q1 = the next 128).
 //   warps 0-3  softmax for Q0 (thread = row = TMEM lane), warps 4-7 softmax for Q1,
 //   warp 8     TMA producer (Q pair, then K_j, V_j per key tile into an NSTAGE ring),
@@ -23,6 +23,7 @@
 #pragma once
 #include "ra_schedule.h"
 #include "ra_sm100.cuh"
+#include "ra_work.cuh"
 
 namespace ra {
 namespace fwd {
@@ -56,8 +57,10 @@ struct Layout {
   // barrier indices
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_KV_FULL = 2, B_KV_EMPTY = B_KV_FULL + NSTAGE,
                        B_S_FULL = B_KV_EMPTY + NSTAGE, B_P_READY = B_S_FULL + NQ, B_O_FINAL = B_P_READY + NQ,
-                       B_DRAIN = B_O_FINAL + NQ, NUM_BARS = B_DRAIN + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+                       B_DRAIN = B_O_FINAL + NQ, B_WQ_FULL = B_DRAIN + 1, B_WQ_EMPTY = B_WQ_FULL + 2,
+                       NUM_BARS = B_WQ_EMPTY + 2;
+  static constexpr uint32_t WQ_CONSUMERS = 1 + 8;   // MMA thread + one arrival per softmax warp
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, item ring[2]
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;           // room to align the base to 1024 B
   // TMEM columns of S_t (P_t aliases its first 64) and of O_t.
@@ -69,15 +72,23 @@ struct Params {
   int BH, S, D, causal;
   int n_pairs;        // ceil(S / ROWS)
   int n_items;        // BH * n_pairs
+  int hgroup;         // heads whose items are interleaved (L2 reuse of K, V)
+  int work_slot;      // this launch's work counter
   float scale_log2;   // softmax scale * log2(e)
   __nv_bfloat16* o;   // [BH][S][HD]
   float* lse;         // [BH][S]
 };
 
-// Work item w -> (bh, pair).  Causal: longest items (last query tiles) first.
+// Work item w -> (bh, pair).  Heads are taken in groups of p.hgroup (all heads by default);
+// inside a group items go pair by pair, causal: the last query tiles (longest items) first,
+// so the CTAs that fetch items dynamically finish together.
 __device__ __forceinline__ void item_coords(int w, const Params& p, int& bh, int& pair) {
-  const int rank = w / p.BH;
-  bh = w - rank * p.BH;
+  const int per_group = p.hgroup * p.n_pairs;
+  const int g = w / per_group;
+  const int gsize = min(p.hgroup, p.BH - g * p.hgroup);
+  const int idx = w - g * per_group;
+  const int rank = idx / gsize;
+  bh = g * p.hgroup + (idx - rank * gsize);
   pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
 }
 
@@ -91,7 +102,7 @@ __device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
 // ------------------------------------------------------------------ producer (1 thread)
 template <int HD>
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                         const Params& p, uint32_t sbase, volatile int* abort_flag) {
+                         const Params& p, uint32_t sbase, volatile int* wq, volatile int* abort_flag) {
   using L = Layout<HD>;
   const uint32_t bars = sbase + L::BAR_OFF;
   auto bar = [&](int i) { return bars + 8u * i; };
@@ -101,7 +112,12 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
   int q_issued = 0;
   uint32_t q_parity = 0;
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  int w = work_fetch(p.work_slot);
+  for (;;) {
+    if (!ring.push(w, abort_flag)) { ok = false; break; }
+    if (w >= p.n_items) break;
+    const int w_next = work_fetch(p.work_slot);   // in flight while this item's loads issue
     int bh, pair;
     item_coords(w, p, bh, pair);
     const int q0 = pair * ROWS;
@@ -135,7 +151,10 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
       }
       if (!ok) break;
     }
+    if (!ok) break;
+    w = w_next;
   }
+  work_done(p.work_slot);
   if (!ok) {  // let every copy this CTA started land before the CTA can exit
     for (int s = 0; s < NSTAGE; ++s)
       if (issued & (1u << s)) drain_wait(bar(L::B_KV_FULL + s), (issued_parity >> s) & 1u);
@@ -173,7 +192,7 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, i
 }
 
 template <int HD>
-__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
   using L = Layout<HD>;
   const uint32_t bars = sbase + L::BAR_OFF;
   auto bar = [&](int i) { return bars + 8u * i; };
@@ -181,7 +200,11 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
   uint32_t phase = 0, q_phase = 0;
   uint32_t p_phase[NQ] = {0, 0};
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (;;) {
+    int w;
+    if (!ring.pop(w, abort_flag)) { ok = false; break; }
+    if (w >= p.n_items) break;
     int bh, pair;
     item_coords(w, p, bh, pair);
     if (!mbar_wait(bar(L::B_Q_FULL), q_phase, abort_flag)) { ok = false; break; }
@@ -235,7 +258,8 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
 
 // ------------------------------------------------------------------ softmax (128 threads)
 template <int HD>
-__device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq,
+                           volatile int* abort_flag) {
   using L = Layout<HD>;
   const uint32_t bars = sbase + L::BAR_OFF;
   auto bar = [&](int i) { return bars + 8u * i; };
@@ -248,7 +272,11 @@ __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem
   const float sl2 = p.scale_log2;
   uint32_t s_phase = 0, o_phase = 0;
 
-  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (;;) {
+    int w;
+    if (!ring.pop_warp(w, abort_flag)) return;
+    if (w >= p.n_items) break;
     int bh, pair;
     item_coords(w, p, bh, pair);
     const int q_tile0 = pair * ROWS + t * BM;
@@ -359,13 +387,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  volatile int* wq = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
     const uint32_t bars = sbase + L::BAR_OFF;
     for (int i = 0; i < L::NUM_BARS; ++i) {
       const bool p_ready = (i >= L::B_P_READY && i < L::B_P_READY + NQ);
-      mbar_init(bars + 8u * i, p_ready ? BM : 1);
+      const bool wq_empty = (i >= L::B_WQ_EMPTY && i < L::B_WQ_EMPTY + 2);
+      mbar_init(bars + 8u * i, p_ready ? BM : (wq_empty ? L::WQ_CONSUMERS : 1));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -387,15 +417,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp >= 8) {
     regs_lower<REGS_OTHER>();
     if (warp == WARP_TMA) {
-      if ((threadIdx.x & 31) == 0) producer<HD>(&tm_q, &tm_k, &tm_v, p, sbase, abort_flag);
+      if ((threadIdx.x & 31) == 0) producer<HD>(&tm_q, &tm_k, &tm_v, p, sbase, wq, abort_flag);
       __syncwarp();
     } else if (warp == WARP_MMA) {
-      if ((threadIdx.x & 31) == 0) mma_issuer<HD>(p, sbase, tmem, abort_flag);
+      if ((threadIdx.x & 31) == 0) mma_issuer<HD>(p, sbase, tmem, wq, abort_flag);
       __syncwarp();
     }
   } else {
     regs_raise<REGS_SOFTMAX>();
-    softmax_wg<HD>(warp >> 2, p, sbase, tmem, abort_flag);
+    softmax_wg<HD>(warp >> 2, p, sbase, tmem, wq, abort_flag);
   }
 
   tc_fence_before();

@@ -54,6 +54,7 @@ EncodeTiledFn encode_fn() {
 
 struct DevInfo {
   int sm_count = 0;
+  std::atomic<unsigned> next_work_slot{0};   // round robin over the kernels' work counters
   bool ok = false;          // compute capability 10.0
   bool fwd_attr[2] = {false, false};
   bool bwd_attr = false;
@@ -94,16 +95,19 @@ DevInfo* dev_info(int* status) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 3-D tensor map over a [BH][S][Dh] bf16 tensor: box = 64 columns (128 B) x `box_rows` rows
-// x 1 head, 128-byte swizzle, zero fill outside [0, S) so tiles never read the next head.
-int make_map(CUtensorMap* map, const void* base, long long BH, int S, int Dh, int box_rows) {
+// 3-D tensor map over a [BH][S][Dh] tensor (bf16, or fp32 when `f32`): box = 128 bytes of
+// columns x `box_rows` rows x 1 head, 128-byte swizzle, zero fill outside [0, S) so tiles
+// never read the next head (and stores/reductions there are dropped).
+int make_map(CUtensorMap* map, const void* base, long long BH, int S, int Dh, int box_rows, bool f32 = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cuda_fail(-1, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+  const cuuint64_t esz = f32 ? 4 : 2;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Dh), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Dh) * 2, static_cast<cuuint64_t>(S) * Dh * 2};
-  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Dh) * esz, static_cast<cuuint64_t>(S) * Dh * esz};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  const CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                         const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? RA_OK : cuda_fail(static_cast<int>(r), "cuTensorMapEncodeTiled");
@@ -118,6 +122,12 @@ int check_shape(int B, int H, int S, int Dh, int D) {
   if (BH > INT_MAX / 2) return RA_ERR_SHAPE;
   if (static_cast<double>(BH) * S * Dh > 9.0e18 / 4) return RA_ERR_SHAPE;
   return RA_OK;
+}
+
+// Heads whose per-head streamed operands (`bytes_per_head`) fit together in ~48 MiB of L2.
+int heads_per_l2_group(long long BH, long long bytes_per_head) {
+  const long long g = (48ll << 20) / (bytes_per_head > 0 ? bytes_per_head : 1);
+  return static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
 }
 
 int launch_status() {
@@ -147,6 +157,10 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   const long long items = BH * p.n_pairs;
   if (items > INT_MAX) return RA_ERR_SHAPE;
   p.n_items = static_cast<int>(items);
+  // All heads interleaved: with dynamic scheduling this measured best per cycle at S = 16K
+  // and 32K; grouping heads for L2 reuse pays off in the backward only.
+  p.hgroup = static_cast<int>(BH);
+  p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -228,6 +242,8 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = make_map(&mk, k, BH, S, rb::HD, rb::BM)) != RA_OK) return st;
   if ((st = make_map(&mv, v, BH, S, rb::HD, rb::BM)) != RA_OK) return st;
   if ((st = make_map(&mdo, dO, BH, S, rb::HD, rb::BQ)) != RA_OK) return st;
+  CUtensorMap mdq;   // fp32 accumulator, 32-column boxes for the reduce-adds
+  if ((st = make_map(&mdq, dq_acc, BH, S, rb::HD, rb::BQ, true)) != RA_OK) return st;
   rb::Params p;
   p.BH = static_cast<int>(BH);
   p.S = S;
@@ -238,6 +254,8 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   const long long items = BH * p.n_kt;
   if (items > INT_MAX) return RA_ERR_SHAPE;
   p.n_items = static_cast<int>(items);
+  p.hgroup = heads_per_l2_group(BH, 4ll * S * rb::HD);   // Q + dO bytes of one head
+  p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.lse2 = lse2;
@@ -252,7 +270,7 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
     di->bwd_attr = true;
   }
   const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
-  rb::bwd_kernel<<<grid, rb::NUM_THREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  rb::bwd_kernel<<<grid, rb::NUM_THREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
   if ((st = launch_status()) != RA_OK) return st;
 
   // 3. dQ = scale * accumulator -> bf16
