@@ -208,6 +208,14 @@ RA_API int ring_attn_device_status(ra_stream stream);
  */
 RA_API int ring_attn_last_cuda_error(const char** site);
 
+/*
+ * ring_attn_exp2_check -- numerical self-check of the two base-2 exponentials the softmax
+ * kernels use (no counterpart on the pages): for i < n, y_fma[i] = the polynomial evaluation on
+ * the FMA pipes (relative error <= 1.0e-4 for x in [-126, 8]) and y_mufu[i] = the hardware
+ * ex2.approx unit.  x, y_fma, y_mufu are device float32 arrays of n elements.
+ */
+RA_API int ring_attn_exp2_check(const float* x, float* y_fma, float* y_mufu, long long n, ra_stream stream);
+
 /* Static English text for a status code. */
 RA_API const char* ring_attn_strerror(int code);
 

@@ -8,8 +8,9 @@
 //   dS = P * (dP - Delta), dQ = scale dS K, dK = scale dS^T Q.
 //
 // Three kernels:
-//   bwd_pre     Delta (fp32), lse * log2(e) (fp32), both padded per head to a multiple of
-//               128 rows, and a zeroed fp32 dQ accumulator (HBM-bound).
+//   bwd_pre     -Delta (fp32) and -lse * log2(e) (fp32), both padded per head to a multiple
+//               of 128 rows, and a zeroed fp32 dQ accumulator (HBM-bound).  Stored negated
+//               so the key-row warpgroup's elementwise work is one packed add/FMA per pair.
 //   bwd_kernel  key/value-stationary: one CTA per (head, 128-key tile) at a time, visiting
 //               the query tiles that can see the key tile in ring order (ring step t brings
 //               the key/value block j to the position of query block (j + t) mod D, step 0
@@ -49,6 +50,10 @@ constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr uint32_t REGS_LAUNCH = 168, REGS_WG0 = 248, REGS_OTHER = 88;
 static_assert(REGS_WG0 - REGS_LAUNCH <= REGS_LAUNCH - REGS_OTHER, "register split exceeds the pool");
 constexpr uint32_t TMEM_COLS = 512;
+// Of every 8 columns of P, 2 x this many exponentials run on the FMA pipes (exp2_fma2).
+#ifndef RA_BWD_EXP2_FMA_PER4
+#define RA_BWD_EXP2_FMA_PER4 1
+#endif
 constexpr uint32_t COL_S = 0, COL_DQ0 = 64, COL_DP = 128, COL_DS = 128, COL_DQ1 = 192, COL_DV = 256, COL_DK = 384;
 
 struct Layout {
@@ -80,8 +85,8 @@ struct Params {
   int work_slot;         // this launch's work counter
   float scale_log2;      // scale * log2(e)
   float scale;
-  const float* lse2;     // [BH][S_pad] lse * log2(e), +inf in padding
-  const float* delta;    // [BH][S_pad]
+  const float* lse2;     // [BH][S_pad] -lse * log2(e), -inf in padding
+  const float* delta;    // [BH][S_pad] -Delta
   float* dq_acc;         // [BH][S][HD] fp32
   __nv_bfloat16* dk;     // [BH][S][HD]
   __nv_bfloat16* dv;
@@ -301,12 +306,27 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
           tmem_ld32(lane_base + COL_S + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
         tmem_ld_wait();
 #pragma unroll
+        const float2 sl2x2 = make_float2(sl2, sl2);
+#pragma unroll
         for (int c = 0; c < BQ; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
-          pv[c + 0] = ex2_approx(fmaf(__uint_as_float(r[c + 0]), sl2, -l4.x));
-          pv[c + 1] = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, -l4.y));
-          pv[c + 2] = ex2_approx(fmaf(__uint_as_float(r[c + 2]), sl2, -l4.z));
-          pv[c + 3] = ex2_approx(fmaf(__uint_as_float(r[c + 3]), sl2, -l4.w));
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);   // -lse * log2(e)
+          const float2 xa = __ffma2_rn(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2x2,
+                                       make_float2(l4.x, l4.y));
+          const float2 xb = __ffma2_rn(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl2x2,
+                                       make_float2(l4.z, l4.w));
+          float2 pa, pb;
+          if (((c >> 2) & 1) < RA_BWD_EXP2_FMA_PER4) {
+            pa = exp2_fma2(xa);
+          } else {
+            pa.x = ex2_approx(xa.x);
+            pa.y = ex2_approx(xa.y);
+          }
+          pb.x = ex2_approx(xb.x);
+          pb.y = ex2_approx(xb.y);
+          pv[c] = pa.x;
+          pv[c + 1] = pa.y;
+          pv[c + 2] = pb.x;
+          pv[c + 3] = pb.y;
         }
       }
       if (masked) {
@@ -340,10 +360,10 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float2 dl = *reinterpret_cast<const float2*>(dlt + 32 * ch + c);
-          const float a = pv[32 * ch + c] * (__uint_as_float(d[c]) - dl.x);
-          const float b = pv[32 * ch + c + 1] * (__uint_as_float(d[c + 1]) - dl.y);
-          pk[c >> 1] = pack_bf16x2(a, b);
+          const float2 ndl = *reinterpret_cast<const float2*>(dlt + 32 * ch + c);   // -Delta
+          const float2 g = __fmul2_rn(make_float2(pv[32 * ch + c], pv[32 * ch + c + 1]),
+                                      __fadd2_rn(make_float2(__uint_as_float(d[c]), __uint_as_float(d[c + 1])), ndl));
+          pk[c >> 1] = pack_bf16x2(g.x, g.y);
         }
         tmem_st16(lane_base + COL_DS + 16 * ch, pk);
         // shared dS: queries 32ch..32ch+31 = half ch/2, 16-B chunks 4(ch&1) .. +3
@@ -525,7 +545,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ------------------------------------------------------------------ preprocess / convert
 constexpr int PRE_WARPS = 8;
 
-// One warp per padded row: Delta = sum_d dO * O, lse2 = lse * log2(e) (+inf and 0 in the
+// One warp per padded row: -Delta = -sum_d dO * O and -lse * log2(e) (0 and -inf in the
 // padding rows), and the row of the fp32 dQ accumulator cleared.
 __global__ void __launch_bounds__(PRE_WARPS * 32)
     bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
@@ -539,7 +559,7 @@ __global__ void __launch_bounds__(PRE_WARPS * 32)
   if (s >= S) {
     if (lane == 0) {
       delta[prow] = 0.f;
-      lse2[prow] = INFINITY;
+      lse2[prow] = -INFINITY;
     }
     return;
   }
@@ -560,8 +580,8 @@ __global__ void __launch_bounds__(PRE_WARPS * 32)
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   reinterpret_cast<float4*>(dq_acc + row * HD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane == 0) {
-    delta[prow] = acc;
-    lse2[prow] = lse[row] * 1.4426950408889634f;
+    delta[prow] = -acc;
+    lse2[prow] = -lse[row] * 1.4426950408889634f;
   }
 }
 

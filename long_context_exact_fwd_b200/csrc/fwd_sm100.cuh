@@ -43,6 +43,13 @@ constexpr uint32_t REGS_LAUNCH = 168, REGS_SOFTMAX = 208, REGS_OTHER = 88;
 static_assert(2 * (REGS_SOFTMAX - REGS_LAUNCH) <= REGS_LAUNCH - REGS_OTHER, "register split exceeds the pool");
 static_assert(NUM_THREADS * REGS_LAUNCH <= 65536, "launch register budget");
 constexpr float RESCALE_LOG2 = 8.0f;
+// Of every 4 exponential pairs of a row, this many are evaluated on the FMA pipes
+// (exp2_fma2) and the rest on MUFU.  Measured on B200 at S = 16K and 32K: 0 is fastest for
+// this kernel (the softmax warps are issue-bound, and the polynomial costs more issue slots
+// than the MUFU cycles it saves), so the knob stays at 0.
+#ifndef RA_FWD_EXP2_FMA_PER4
+#define RA_FWD_EXP2_FMA_PER4 0
+#endif
 constexpr uint32_t TMEM_COLS = 512;
 
 template <int HD>
@@ -305,9 +312,16 @@ __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      float mx;
+      {  // row max: four independent chains of three-input maxima
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        for (int c = 0; c < BN; c += 8)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            m4[j] = fmax3(m4[j], __uint_as_float(s[c + 2 * j]), __uint_as_float(s[c + 2 * j + 1]));
+        mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+      }
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_ref, m_tile);
       const bool raise = m_new > m_ref + RESCALE_LOG2;   // false while nothing is visible
@@ -330,23 +344,34 @@ __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem
         m_ref = m_new;
       }
       const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      float rs = 0.f;
+      const float2 sl2x2 = make_float2(sl2, sl2), nref2 = make_float2(neg_ref, neg_ref);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // two halves of 64 keys -> 32 packed columns each
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[64 * h + 2 * c]), sl2, neg_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[64 * h + 2 * c + 1]), sl2, neg_ref));
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[64 * h + 2 * c]),
+                                                  __uint_as_float(s[64 * h + 2 * c + 1])), sl2x2, nref2);
+          float2 pp;
+          if ((c & 3) < RA_FWD_EXP2_FMA_PER4) {
+            pp = exp2_fma2(x);
+          } else {
+            pp.x = ex2_approx(x.x);
+            pp.y = ex2_approx(x.y);
+          }
+          if (c & 1)
+            acc1 = __fadd2_rn(acc1, pp);
+          else
+            acc0 = __fadd2_rn(acc0, pp);
+          pk[c] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st32(tS + 32 * h, pk);
       }
-      l += rs;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::B_P_READY + t));
+      mbar_arrive(bar(L::B_P_READY + t));   // the row sum is not needed by the MMA
+      l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
     }
     // epilogue: O = O_acc / l (bf16), LSE = (m_ref + log2 l) * ln 2
     if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_O_FINAL + t), o_phase, abort_flag))) return;

@@ -283,6 +283,43 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA/ALU pipes, for spreading exponentials between MUFU and the FMA units.
+// Cody-Waite split x = n + f with n = rint(x), read from the low mantissa bits of
+// x + 1.5 * 2^23, and f in [-1/2, 1/2]; 2^f from a cubic 1 + c1 f + c2 f^2 + c3 f^3 whose
+// coefficients were fitted for this library by relative-error minimax on [-1/2, 1/2]
+// (Lawson's iteratively reweighted least squares, p(0) = 1); 2^n is added into the exponent
+// field.  Maximum relative error 1.0e-4 for x in [-126, 8], below the bf16 rounding that P
+// receives.  Inputs below -126 (including -inf) return 2^-126.
+constexpr float EXP2_C1 = 0.6932829022407532f, EXP2_C2 = 0.2422105371952057f, EXP2_C3 = 0.05500870570540428f;
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  const float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two lanes of exp2_fma with packed f32x2 arithmetic (same polynomial, same bound).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
+  p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
   return *reinterpret_cast<uint32_t*>(&v);

@@ -282,9 +282,28 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   return launch_status();
 }
 
+__global__ void exp2_check_kernel(const float* __restrict__ x, float* __restrict__ y_fma, float* __restrict__ y_mufu,
+                                  long long n) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) {
+    y_fma[i] = ra::exp2_fma(x[i]);
+    y_mufu[i] = ra::ex2_approx(x[i]);
+  }
+}
+
 }  // namespace
 
 extern "C" {
+
+int ring_attn_exp2_check(const float* x, float* y_fma, float* y_mufu, long long n, ra_stream stream) {
+  if (!x || !y_fma || !y_mufu || n <= 0) return RA_ERR_ARG;
+  int st = RA_OK;
+  if (!dev_info(&st)) return st;
+  const long long blocks = (n + 255) / 256;
+  if (blocks > INT_MAX) return RA_ERR_SHAPE;
+  exp2_check_kernel<<<static_cast<int>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_fma, y_mufu, n);
+  return launch_status();
+}
 
 int ring_attn_version(void) { return RA_VERSION; }
 

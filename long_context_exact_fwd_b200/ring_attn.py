@@ -49,6 +49,7 @@ _bwd_visit_tiles = _sig("ring_attn_bwd_visit_tiles", _i, _i, _i, _i, _i, _i, _ip
 _launch_count = _sig("ring_attn_launch_count", ctypes.c_ulonglong)
 _bwd_noalloc = _sig("ring_attn_bwd_noalloc", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _noalloc_max = _sig("ring_attn_bwd_noalloc_max_bytes", _sz)
+_exp2_check = _sig("ring_attn_exp2_check", _i, _vp, _vp, _vp, ctypes.c_longlong, _vp)
 
 
 class RingAttnError(RuntimeError):
@@ -223,6 +224,15 @@ def bwd_visit_tiles(S: int, D: int, causal: bool, k0: int, rows: int = 128) -> L
     if n < 0:
         raise RingAttnError(-n, "ring_attn_bwd_visit_tiles")
     return list(buf[:n])
+
+
+def exp2_check(x: torch.Tensor, stream=None):
+    """Evaluate the kernels' two base-2 exponentials on x (float32, CUDA): returns
+    (polynomial on the FMA pipes, hardware ex2.approx)."""
+    _need(x, "x", torch.float32)
+    y1, y2 = torch.empty_like(x), torch.empty_like(x)
+    _check(_exp2_check(x.data_ptr(), y1.data_ptr(), y2.data_ptr(), x.numel(), _stream(stream)), "ring_attn_exp2_check")
+    return y1, y2
 
 
 def launch_count() -> int:

@@ -202,3 +202,21 @@ def test_ring_steps_as_separate_calls_then_merged(ra, causal):
     O, L = oracle.attn_fwd_heads(inp["q"], inp["k"], inp["v"], causal)
     assert_close_bf16(o.float().cpu().numpy(), O)
     assert_lse(lse.cpu().numpy(), L)
+
+
+def test_fma_pipe_exp2_against_exp2_and_its_bound(ra):
+    """The polynomial 2^x spread onto the FMA pipes stays within its 1.0e-4 relative bound
+    of the exact value (float64) on [-126, 8], returns exactly-representable powers of two
+    at integers within the bound, and maps -inf to a negligible 2^-126."""
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1 << 20), torch.arange(-126, 9, dtype=torch.float32),
+                   torch.tensor([float("-inf"), -1000.0])]).cuda()
+    y_fma, y_mufu = ra.exp2_check(x)
+    assert ra.device_status() == 0
+    xs = x[:-2].double().cpu()
+    exact = torch.exp2(xs)
+    rel = ((y_fma[:-2].double().cpu() - exact).abs() / exact)
+    assert rel.max().item() <= 1.05e-4, rel.max().item()
+    rel_hw = ((y_mufu[:-2].double().cpu() - exact).abs() / exact)
+    assert rel_hw.max().item() <= 2e-6              # hardware unit, for reference
+    assert y_fma[-2].item() <= 1.2e-38 and y_fma[-1].item() <= 1.2e-38
+    assert y_fma[-2].item() >= 0.0 and y_fma[-1].item() >= 0.0
