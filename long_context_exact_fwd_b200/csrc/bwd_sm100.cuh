@@ -18,19 +18,24 @@
 //               the fp32 accumulator by TMA bulk reduce-add.
 //   bwd_convert dQ = scale * accumulator -> bf16 (HBM-bound).
 //
-// bwd_kernel CTA (384 threads):
-//   warpgroup 0  thread = key row: P^T, dS^T (bf16) into TMEM and dS into shared memory;
-//                final dK, dV epilogue.
-//   warpgroup 1  thread = query row: reads dQ from TMEM, stages it (fp32, 128-B swizzled
-//                32-column boxes) in the dS buffer once the dQ MMAs have consumed dS, and one
-//                thread issues TMA reduce-adds into the fp32 accumulator.
-//   warp 8       TMA producer: K, V once per item; Q, dO, lse2, Delta per query tile (2 stages).
-//   warp 9       TMEM allocator + tcgen05.mma issuer.
-// TMEM (512 columns): [0,128) S^T, P^T (bf16) in [0,64), dQ[:, 0:64] in [64,128);
-//   [128,256) dP^T, dS^T (bf16) in [128,192), dQ[:, 64:128] in [192,256);
-//   [256,384) dV; [384,512) dK.
-// MMAs per query tile (M = 128, K = 128 each): S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
-//   dK += dS^T Q, dQ(two N = 64 halves) = dS K.
+// bwd_kernel CTA (512 threads):
+//   warpgroups 0, 1  thread = key row, warpgroup h taking query columns [64h, 64h + 64): P^T,
+//                dS^T (bf16) into TMEM and dS into shared memory; final dK, dV epilogue (head
+//                columns [64h, 64h + 64)).  Each writes TMEM only inside columns it has itself
+//                read, so the two never race.
+//   warpgroup 2  thread = query row: reads dQ from TMEM, stages it (fp32, four 128-B swizzled
+//                32-column boxes, 64 KB) over the query tile's own Q/dO stage once dK has read
+//                Q, and one thread issues the TMA reduce-adds into the fp32 accumulator and
+//                then hands the stage back to the producer.
+//   warp 12      TMA producer: K, V once per item; Q, dO, lse2, Delta per query tile (2 stages).
+//   warp 13      TMEM allocator + tcgen05.mma issuer (warps 14, 15 complete warpgroup 3).
+// TMEM (512 columns): [0,128) S^T, then P^T (bf16) of queries 0-63 in [0,32) and of queries
+//   64-127 in [96,128); [128,256) dP^T, then dS^T in [128,160) and [224,256), then dQ once
+//   dK has consumed dS^T; [256,384) dV; [384,512) dK.
+// MMAs per query tile (M = N = K = 128 each, in this order): S^T = K Q^T, dP^T = V dO^T,
+//   dV += P^T dO, dK += dS^T Q, dQ = dS K.  The tensor pipe executes them in issue order, so
+//   a later MMA may overwrite TMEM an earlier one reads: S^T of the next tile is issued right
+//   after dQ (P^T is dead once dV issued), and only its dP^T waits for the dQ readout.
 #pragma once
 #include "ra_schedule.h"
 #include "ra_sm100.cuh"
@@ -43,18 +48,30 @@ constexpr int BM = 128;   // keys per CTA tile (TMEM lanes of S^T, dP^T, dV, dK)
 constexpr int BQ = 128;   // queries per query tile
 constexpr int HD = 128;   // head dimension of this kernel
 constexpr int NSTAGE = 2;
-constexpr int NUM_THREADS = 384;
-constexpr int WARP_TMA = 8, WARP_MMA = 9;
-// Registers: launched at 168.  Warpgroup 2 lowers to 88 (frees 128 x 80); warpgroup 0
-// raises to 248 (takes 128 x 80); warpgroup 1 keeps 168.
-constexpr uint32_t REGS_LAUNCH = 168, REGS_WG0 = 248, REGS_OTHER = 88;
-static_assert(REGS_WG0 - REGS_LAUNCH <= REGS_LAUNCH - REGS_OTHER, "register split exceeds the pool");
+constexpr int NUM_THREADS = 512;
+constexpr int WARP_TMA = 12, WARP_MMA = 13;
+// Registers: launched at 65536 / 512 = 128.  Warpgroup 3 (TMA, MMA, idle) lowers to
+// REGS_OTHER; the key-row warpgroups raise to REGS_KEYS and the dQ warpgroup (128 fp32 dQ
+// values per thread) to REGS_DQ.  The raises must not exceed what warpgroup 3 returns.
+#ifndef RA_BWD_REGS_KEYS
+#define RA_BWD_REGS_KEYS 144
+#define RA_BWD_REGS_DQ 168
+#define RA_BWD_REGS_OTHER 56
+#endif
+constexpr uint32_t REGS_LAUNCH = 128;
+constexpr uint32_t REGS_KEYS = RA_BWD_REGS_KEYS, REGS_DQ = RA_BWD_REGS_DQ, REGS_OTHER = RA_BWD_REGS_OTHER;
+static_assert(2 * (REGS_KEYS - REGS_LAUNCH) + (REGS_DQ - REGS_LAUNCH) <= REGS_LAUNCH - REGS_OTHER,
+              "register split exceeds the pool");
+static_assert(NUM_THREADS * REGS_LAUNCH <= 65536, "launch register budget");
 constexpr uint32_t TMEM_COLS = 512;
 // Of every 8 columns of P, 2 x this many exponentials run on the FMA pipes (exp2_fma2).
 #ifndef RA_BWD_EXP2_FMA_PER4
 #define RA_BWD_EXP2_FMA_PER4 1
 #endif
-constexpr uint32_t COL_S = 0, COL_DQ0 = 64, COL_DP = 128, COL_DS = 128, COL_DQ1 = 192, COL_DV = 256, COL_DK = 384;
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 384;
+// bf16 P^T / dS^T of query columns [64h, 64h + 64): TMEM columns [base, base + 32)
+__host__ __device__ constexpr uint32_t col_p(int h) { return h ? 96u : 0u; }
+__host__ __device__ constexpr uint32_t col_ds(int h) { return h ? 224u : 128u; }
 
 struct Layout {
   static constexpr int SUB_BYTES = 128 * 128;          // 128 rows x 128 B (64 bf16)
@@ -69,9 +86,9 @@ struct Layout {
   static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_QD_FULL = 2, B_QD_EMPTY = B_QD_FULL + NSTAGE,
                        B_S_FULL = B_QD_EMPTY + NSTAGE, B_DP_FULL = B_S_FULL + 1, B_P_READY = B_DP_FULL + 1,
                        B_DS_READY = B_P_READY + 1, B_DQ_FULL = B_DS_READY + 1, B_DQ_FREE = B_DQ_FULL + 1,
-                       B_ACC_FULL = B_DQ_FREE + 1, B_DS_FREE = B_ACC_FULL + 1, B_DRAIN = B_DS_FREE + 1,
+                       B_ACC_FULL = B_DQ_FREE + 1, B_DK_DONE = B_ACC_FULL + 1, B_DRAIN = B_DK_DONE + 1,
                        B_WQ_FULL = B_DRAIN + 1, B_WQ_EMPTY = B_WQ_FULL + 2, NUM_BARS = B_WQ_EMPTY + 2;
-  static constexpr uint32_t WQ_CONSUMERS = 1 + 8;   // MMA thread + one arrival per warp of warpgroups 0, 1
+  static constexpr uint32_t WQ_CONSUMERS = 1 + 12;   // MMA thread + one arrival per warp of warpgroups 0-2
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, item ring[2]
   static constexpr int BYTES = MISC_OFF + 16;
 };
@@ -181,23 +198,25 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uin
   }
 }
 
-__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
-  // D[128 x 128] (+)= A[128 x 128] (TMEM, bf16) * B[128 x 128] (smem, MN-major: rows = K)
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_smem,
+                                           bool accumulate) {
+  // D[128 x 128] (+)= A[128 x 128] (TMEM, bf16; K = 0-63 at a_lo, 64-127 at a_hi)
+  //                   * B[128 x 128] (smem, MN-major: rows = K)
   constexpr uint32_t IDESC = idesc_bf16_f32(128, HD, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < BQ / 16; ++kk)
-    umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC,
-            (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, (kk < 4 ? a_lo : a_hi) + (kk & 3) * 8, sdesc_sw128(b_smem + kk * 2048, Layout::SUB_BYTES, 1024),
+            IDESC, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-__device__ __forceinline__ void mma_dq_half(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_half_smem) {
-  // dQ[:, h] [128 q x 64] = dS [128 q x 128 k] (MN-major: q contiguous, two 64-q halves)
-  //                        * K[:, h] [128 k x 64] (MN-major: rows = K)
-  constexpr uint32_t IDESC = idesc_bf16_f32(128, 64, 1, 1);
+__device__ __forceinline__ void mma_dq(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_smem) {
+  // dQ [128 q x 128] = dS [128 q x 128 k] (MN-major: q contiguous, two 64-q halves)
+  //                   * K [128 k x 128] (MN-major: rows = K, two 64-column halves)
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, HD, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < BM / 16; ++kk)
     umma_ss(d_tmem, sdesc_sw128(ds_smem + kk * 2048, Layout::SUB_BYTES, 1024),
-            sdesc_sw128(k_half_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC, kk > 0 ? 1u : 0u);
+            sdesc_sw128(k_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC, kk > 0 ? 1u : 0u);
 }
 
 __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
@@ -225,26 +244,26 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
       const uint32_t st = sbase + L::STAGE_OFF + s * L::STAGE_BYTES;
       if (!mbar_wait(bar(L::B_QD_FULL + s), phase, abort_flag)) { ok = false; break; }
       advance(stage, phase);
-      if (dq_pending) {  // S^T and dP^T overwrite the columns the dQ readout is reading
-        if (!mbar_wait(bar(L::B_DQ_FREE), dqf_phase, abort_flag)) { ok = false; break; }
-        dqf_phase ^= 1u;
-      }
       tc_fence_after();
       mma_kmajor(tmem + COL_S, sbase + L::K_OFF, st + L::STAGE_Q, true);     // S^T = K Q^T
       tc_commit(bar(L::B_S_FULL));
+      if (dq_pending) {  // dP^T overwrites the columns the previous tile's dQ readout reads
+        if (!mbar_wait(bar(L::B_DQ_FREE), dqf_phase, abort_flag)) { ok = false; break; }
+        dqf_phase ^= 1u;
+        tc_fence_after();
+      }
       mma_kmajor(tmem + COL_DP, sbase + L::V_OFF, st + L::STAGE_DO, true);   // dP^T = V dO^T
       tc_commit(bar(L::B_DP_FULL));
       if (!mbar_wait(bar(L::B_P_READY), p_phase, abort_flag)) { ok = false; break; }
       p_phase ^= 1u;
       tc_fence_after();
-      mma_tmem_a(tmem + COL_DV, tmem + COL_S, st + L::STAGE_DO, n > 0);     // dV += P^T dO
+      mma_tmem_a(tmem + COL_DV, tmem + col_p(0), tmem + col_p(1), st + L::STAGE_DO, n > 0);   // dV += P^T dO
       if (!mbar_wait(bar(L::B_DS_READY), ds_phase, abort_flag)) { ok = false; break; }
       ds_phase ^= 1u;
       tc_fence_after();
-      mma_tmem_a(tmem + COL_DK, tmem + COL_DS, st + L::STAGE_Q, n > 0);     // dK += dS^T Q
-      tc_commit(bar(L::B_QD_EMPTY + s));                                       // Q, dO, lse2, Delta free
-      mma_dq_half(tmem + COL_DQ0, sbase + L::DS_OFF, sbase + L::K_OFF);
-      mma_dq_half(tmem + COL_DQ1, sbase + L::DS_OFF, sbase + L::K_OFF + L::SUB_BYTES);
+      mma_tmem_a(tmem + COL_DK, tmem + col_ds(0), tmem + col_ds(1), st + L::STAGE_Q, n > 0);   // dK += dS^T Q
+      tc_commit(bar(L::B_DK_DONE));   // Q and dO of this stage no longer read by the tensor core
+      mma_dq(tmem + COL_DQ, sbase + L::DS_OFF, sbase + L::K_OFF);                 // dQ = dS K
       tc_commit(bar(L::B_DQ_FULL));
       dq_pending = true;
     }
@@ -256,7 +275,8 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
   drain_wait(bar(L::B_DRAIN), 0);
 }
 
-// ------------------------------------------------------------------ warpgroup 0: P^T, dS^T, epilogue
+// ------------------------------------------------------------------ warpgroups 0, 1: P^T, dS^T, epilogue
+template <int half>
 __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem, volatile int* wq,
                             volatile int* abort_flag) {
   using L = Layout;
@@ -264,18 +284,19 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
   const int lane = threadIdx.x & 31;
   const int quarter = (threadIdx.x >> 5) & 3;
   const int row = quarter * 32 + lane;   // key row within the tile
+  constexpr int qc0 = 64 * half;         // this warpgroup's first query column
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-  const float sl2 = p.scale_log2;
+  const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
   int stage = 0;
-  uint32_t phase = 0, s_phase = 0, dp_phase = 0, acc_phase = 0, dsf_phase = 0;
-  // dS row of this thread in the MN-major shared tile: half h (queries 64h..64h+63), 16-B
-  // chunk c of the 128-B row goes to chunk c ^ (row & 7) (128-byte swizzle).
-  uint8_t* ds_row = smem + L::DS_OFF + row * 128;
+  uint32_t phase = 0, s_phase = 0, dp_phase = 0, acc_phase = 0;
+  // this thread's dS row in the MN-major shared tile: queries [qc0, qc0 + 64) form half
+  // `half`; 16-B chunk j of the 128-B row is stored at chunk j ^ (row & 7) (128-B swizzle)
+  uint8_t* ds_row = smem + L::DS_OFF + half * L::SUB_BYTES + row * 128;
   const int sw = row & 7;
 
   ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
   for (;;) {
-    int w;
+    int w = 0;
     if (!ring.pop_warp(w, abort_flag)) return;
     if (w >= p.n_items) break;
     int bh, kt;
@@ -284,32 +305,32 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
     RingQTiles it;
     it.init(p.S, p.D, p.causal, kt * BM, BQ);
     for (int qt = it.next(); qt >= 0; qt = it.next()) {
-      const float* lse2 = reinterpret_cast<const float*>(smem + L::STAGE_OFF + stage * L::STAGE_BYTES + L::STAGE_LSE);
-      const float* dlt = reinterpret_cast<const float*>(smem + L::STAGE_OFF + stage * L::STAGE_BYTES + L::STAGE_DELTA);
-      // lse2 / Delta arrive by bulk copy on the stage's full barrier: observe it directly
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QD_FULL + stage), phase, abort_flag))) return;
-      advance(stage, phase);
-      const int q0 = qt * BQ;
-      // visible queries of this key row: [lo, hi) in tile coordinates
+      const uint8_t* stg = smem + L::STAGE_OFF + stage * L::STAGE_BYTES;
+      const float* nlse2 = reinterpret_cast<const float*>(stg + L::STAGE_LSE) + qc0;   // -lse * log2(e)
+      const float* ndlt = reinterpret_cast<const float*>(stg + L::STAGE_DELTA) + qc0;  // -Delta
+      const int q0 = qt * BQ + qc0;
+      // visible queries of this key row: columns [lo, hi) of this warpgroup's 64
       const int lo = p.causal ? k_row - q0 : 0;
       const int hi = (k_row < p.S) ? p.S - q0 : 0;
-      const bool masked = (lo > 0) || (hi < BQ);
+      const bool masked = (lo > 0) || (hi < 64);
 
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_S_FULL), s_phase, abort_flag))) return;
+      // ---- P^T = exp2(S^T * scale * log2e - lse * log2e)
+      // lse2 / Delta arrive by bulk copy on the stage's full barrier: observe it directly
+      bool ok = mbar_wait(bar(L::B_QD_FULL + stage), phase, abort_flag);
+      ok = ok && mbar_wait(bar(L::B_S_FULL), s_phase, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      advance(stage, phase);
       s_phase ^= 1u;
       tc_fence_after();
-      float pv[BQ];
+      float pv[64];
       {
-        uint32_t r[BQ];
-#pragma unroll
-        for (int c = 0; c < BQ / 32; ++c)
-          tmem_ld32(lane_base + COL_S + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+        uint32_t r[64];
+        tmem_ld32(lane_base + COL_S + qc0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(lane_base + COL_S + qc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
 #pragma unroll
-        const float2 sl2x2 = make_float2(sl2, sl2);
-#pragma unroll
-        for (int c = 0; c < BQ; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);   // -lse * log2(e)
+        for (int c = 0; c < 64; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(nlse2 + c);
           const float2 xa = __ffma2_rn(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2x2,
                                        make_float2(l4.x, l4.y));
           const float2 xb = __ffma2_rn(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl2x2,
@@ -331,74 +352,72 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
       }
       if (masked) {
 #pragma unroll
-        for (int c = 0; c < BQ; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c < lo || c >= hi) pv[c] = 0.f;
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {   // P^T (bf16) -> TMEM columns [0, 64)
+      {
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[64 * h + 2 * c], pv[64 * h + 2 * c + 1]);
-        tmem_st32(lane_base + COL_S + 32 * h, pk);
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+        tmem_st32(lane_base + col_p(half), pk);   // inside the S^T columns this warpgroup read
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::B_P_READY));
 
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DP_FULL), dp_phase, abort_flag))) return;
+      // ---- dS^T = P^T * (dP^T - Delta), 32 query columns at a time.  dS^T goes to columns
+      // this warpgroup has already read: warpgroup 1 walks its chunks from the high end.
+      // (the previous tile's dQ MMA, the last reader of the dS buffer, completed before the dQ
+      // readout released the TMEM columns that this tile's dP^T was then written into)
+      ok = mbar_wait(bar(L::B_DP_FULL), dp_phase, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) return;
       dp_phase ^= 1u;
-      // the dS buffer doubles as dQ staging of the previous query tile: wait until its
-      // reduce-adds have read it
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DS_FREE), dsf_phase ^ 1u, abort_flag))) return;
-      dsf_phase ^= 1u;
       tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < BQ / 32; ++ch) {   // 32 queries per chunk
+      for (int i = 0; i < 2; ++i) {
+        const int ch = half ? 1 - i : i;   // chunk = query columns [32 ch, 32 ch + 32) of this half (compile time)
         uint32_t d[32];
-        tmem_ld32(lane_base + COL_DP + 32 * ch, d);
+        tmem_ld32(lane_base + COL_DP + qc0 + 32 * ch, d);
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float2 ndl = *reinterpret_cast<const float2*>(dlt + 32 * ch + c);   // -Delta
+          const float2 nd = *reinterpret_cast<const float2*>(ndlt + 32 * ch + c);
           const float2 g = __fmul2_rn(make_float2(pv[32 * ch + c], pv[32 * ch + c + 1]),
-                                      __fadd2_rn(make_float2(__uint_as_float(d[c]), __uint_as_float(d[c + 1])), ndl));
+                                      __fadd2_rn(make_float2(__uint_as_float(d[c]), __uint_as_float(d[c + 1])), nd));
           pk[c >> 1] = pack_bf16x2(g.x, g.y);
         }
-        tmem_st16(lane_base + COL_DS + 16 * ch, pk);
-        // shared dS: queries 32ch..32ch+31 = half ch/2, 16-B chunks 4(ch&1) .. +3
-        uint8_t* half = ds_row + (ch >> 1) * L::SUB_BYTES;
+        tmem_st16(lane_base + col_ds(half) + 16 * ch, pk);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int chunk = ((ch & 1) * 4 + j) ^ sw;
-          *reinterpret_cast<uint4*>(half + chunk * 16) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(ds_row + (((4 * ch + j) ^ sw) << 4)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       }
       tmem_st_wait();
       fence_proxy_async_smem();   // generic-proxy dS stores -> visible to the tensor core
       tc_fence_before();
       mbar_arrive(bar(L::B_DS_READY));
     }
-    // epilogue: dV, dK (scaled) for this key tile
+    // ---- epilogue: dV, dK (scaled), head columns [64 half, 64 half + 64)
     if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC_FULL), acc_phase, abort_flag))) return;
     acc_phase ^= 1u;
     tc_fence_after();
     const bool row_ok = k_row < p.S;
-    const size_t off = (static_cast<size_t>(bh) * p.S + k_row) * HD;
+    const size_t off = (static_cast<size_t>(bh) * p.S + k_row) * HD + qc0;
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
-      const uint32_t col = which ? COL_DK : COL_DV;
+      const uint32_t col = (which ? COL_DK : COL_DV) + qc0;
       const float mul = which ? p.scale : 1.f;
       __nv_bfloat16* dst_row = (which ? p.dk : p.dv) + off;
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + col + 32 * c, r);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_base + col + 32 * c, rr);
         tmem_ld_wait();
         uint32_t w16[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          w16[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+          w16[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * mul, __uint_as_float(rr[2 * i + 1]) * mul);
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
 #pragma unroll
@@ -409,7 +428,7 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
   }
 }
 
-// ------------------------------------------------------------------ warpgroup 1: dQ readout
+// ------------------------------------------------------------------ warpgroup 2: dQ readout
 __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                               volatile int* wq, volatile int* abort_flag) {
   using L = Layout;
@@ -419,9 +438,9 @@ __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t
   const int row = quarter * 32 + lane;   // query row within the tile
   const bool leader = (threadIdx.x & 127) == 0;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-  uint8_t* stage_row = smem + L::DS_OFF + row * 128;
   const int sw = row & 7;
-  uint32_t phase = 0;
+  uint32_t phase = 0, dk_phase = 0, qphase = 0;
+  int stage = 0;
   bool ok = true;
   ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
   for (;;) {
@@ -442,35 +461,37 @@ __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t
       tc_fence_after();
       uint32_t r[HD];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(lane_base + ((c < 2) ? COL_DQ0 + 32 * c : COL_DQ1 + 32 * (c - 2)),
-                  *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + COL_DQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar(L::B_DQ_FREE));   // dQ is in registers: hand the TMEM columns back
-      // dQ row -> four 32-column fp32 boxes (128 B per row, 128-B swizzle), two per round
-#pragma unroll
-      for (int round = 0; round < 2; ++round) {
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const int c0 = 32 * (2 * round + b);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(stage_row + b * L::SUB_BYTES + ((j ^ sw) << 4)) =
-                make_uint4(r[c0 + 4 * j], r[c0 + 4 * j + 1], r[c0 + 4 * j + 2], r[c0 + 4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (leader) {
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-            tma_reduce_add_3d(tm_dq, sbase + L::DS_OFF + b * L::SUB_BYTES, 32 * (2 * round + b), qt * BQ, bh);
-          bulk_commit();
-          bulk_wait_read_all();
-        }
-        named_bar_sync(1, 128);   // staging may be overwritten
+      // the tile's Q/dO stage becomes staging once dK (the last MMA reading Q) has completed
+      ok = named_bar_and(1, 128, mbar_wait(bar(L::B_DK_DONE), dk_phase, abort_flag));
+      if (!ok) break;
+      dk_phase ^= 1u;
+      const int s_idx = stage;
+      if (++stage == NSTAGE) {
+        stage = 0;
+        qphase ^= 1u;
       }
-      if (leader) mbar_arrive(bar(L::B_DS_FREE));
+      // dQ row -> four 32-column fp32 boxes (128 B per row, 128-B swizzle) over Q and dO
+      uint8_t* st_row = smem + L::STAGE_OFF + s_idx * L::STAGE_BYTES + row * 128;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(st_row + b * L::SUB_BYTES + ((j ^ sw) << 4)) =
+              make_uint4(r[32 * b + 4 * j], r[32 * b + 4 * j + 1], r[32 * b + 4 * j + 2], r[32 * b + 4 * j + 3]);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (leader) {
+        const uint32_t st = sbase + L::STAGE_OFF + s_idx * L::STAGE_BYTES;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_reduce_add_3d(tm_dq, st + b * L::SUB_BYTES, 32 * b, qt * BQ, bh);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(bar(L::B_QD_EMPTY + s_idx));   // the producer may refill this stage
+      }
     }
     if (!ok) break;
   }
@@ -495,9 +516,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
-      const bool many = (i == L::B_P_READY || i == L::B_DS_READY || i == L::B_DQ_FREE);
+      const bool key_rows = (i == L::B_P_READY || i == L::B_DS_READY);   // both key-row warpgroups
       const bool wq_empty = (i >= L::B_WQ_EMPTY && i < L::B_WQ_EMPTY + 2);
-      mbar_init(sbase + L::BAR_OFF + 8u * i, many ? 128 : (wq_empty ? L::WQ_CONSUMERS : 1));
+      const uint32_t count = key_rows ? 256 : (i == L::B_DQ_FREE ? 128 : (wq_empty ? L::WQ_CONSUMERS : 1));
+      mbar_init(sbase + L::BAR_OFF + 8u * i, count);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -518,7 +540,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp >= 8) {
+  if (warp >= 12) {
     regs_lower<REGS_OTHER>();
     if (warp == WARP_TMA) {
       if ((threadIdx.x & 31) == 0) producer(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, wq, abort_flag);
@@ -527,10 +549,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, wq, abort_flag);
       __syncwarp();
     }
-  } else if (warp < 4) {
-    regs_raise<REGS_WG0>();
-    key_rows_wg(p, smem, sbase, tmem, wq, abort_flag);
+  } else if (warp < 8) {
+    regs_raise<REGS_KEYS>();
+    if (warp < 4)
+      key_rows_wg<0>(p, smem, sbase, tmem, wq, abort_flag);
+    else
+      key_rows_wg<1>(p, smem, sbase, tmem, wq, abort_flag);
   } else {
+    regs_raise<REGS_DQ>();
     query_rows_wg(p, &tm_dq, smem, sbase, tmem, wq, abort_flag);
   }
 
