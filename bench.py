@@ -46,6 +46,28 @@ def _dist_env():
     return ws, rank, local
 
 
+def rank_workload(w: Workload, rank: int) -> Workload:
+    """Each rank runs its own seeded replica of the workload (weak scaling)."""
+    return w.with_(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank number over the process group (the identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step: float, steps: int, max_total_ms: float, world: int) -> float:
+    """Whole-job throughput: every rank did `steps` steps of `flops_per_step`; the job took
+    as long as its slowest rank."""
+    return world * flops_per_step * steps / (max_total_ms * 1e-3) / 1e12
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -232,8 +254,7 @@ def run_ours(args, w: Workload):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    wr = w.with_(seed=w.seed + 1000 * rank)
-    host = make_inputs(wr)
+    host = make_inputs(rank_workload(w, rank))
     names = ("q", "k", "v", "do") if w.backward else ("q", "k", "v")
     x = {n: host[n].to(dev) for n in names}
     o = torch.empty_like(x["q"])
@@ -288,10 +309,7 @@ def run_ours(args, w: Workload):
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if w.backward else [0.0] * args.steps
     step_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_total_ms = float(t.item())
+    max_total_ms = max_over_ranks(total_ms, dev)
 
     # end to end through the public API: pinned host inputs in, gradients (or O) back out
     pinned = {n: host[n].pin_memory() for n in names}
@@ -320,16 +338,13 @@ def run_ours(args, w: Workload):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     if ws > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(te.item())
 
     flops_step = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
-    value = ws * flops_step * args.steps / (max_total_ms * 1e-3) / 1e12
-    e2e_value = ws * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = job_tflops(flops_step, args.steps, max_total_ms, ws)
+    e2e_value = job_tflops(flops_step, args.steps, e2e_ms, ws)
 
     if rank == 0:
         peaks, src = _peaks()

@@ -209,6 +209,15 @@ RA_API int ring_attn_device_status(ra_stream stream);
 RA_API int ring_attn_last_cuda_error(const char** site);
 
 /*
+ * ring_attn_wait_selftest -- exercises the bounded-wait failure path every kernel uses (no
+ * counterpart on the pages): one thread waits on an mbarrier that nothing ever arrives on,
+ * gives up after timeout_ns nanoseconds (0 < timeout_ns <= 1e10) and records RA_ERR_TIMEOUT in
+ * the device status word, exactly as a kernel whose pipeline stalled would.  Read it back with
+ * ring_attn_device_status; the context stays usable.
+ */
+RA_API int ring_attn_wait_selftest(long long timeout_ns, ra_stream stream);
+
+/*
  * ring_attn_exp2_check -- numerical self-check of the two base-2 exponentials the softmax
  * kernels use (no counterpart on the pages): for i < n, y_fma[i] = the polynomial evaluation on
  * the FMA pipes (relative error <= 1.0e-4 for x in [-126, 8]) and y_mufu[i] = the hardware

@@ -71,14 +71,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase of parity `parity` of barrier `bar` to complete.
 // `abort_flag` is a CTA-shared word: once any warp of the CTA has timed out, every
 // other waiter returns false promptly instead of running out its own clock.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t timeout_ns = RA_WAIT_TIMEOUT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1; it != 0; ++it) {   // iteration cap 2^32 - 1 on top of the time cap
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 127u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > RA_WAIT_TIMEOUT_NS) break;
+      if (globaltimer() - t0 > timeout_ns) break;
     }
   }
   *abort_flag = 1;

@@ -282,6 +282,19 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   return launch_status();
 }
 
+// One thread waits, through the kernels' own bounded wait, on an mbarrier nothing arrives on.
+__global__ void wait_selftest_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ra::mbar_init(ra::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ra::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ra::mbar_wait(ra::smem_u32(&bar), 0, &abort_flag, timeout_ns);
+}
+
 __global__ void exp2_check_kernel(const float* __restrict__ x, float* __restrict__ y_fma, float* __restrict__ y_mufu,
                                   long long n) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -294,6 +307,14 @@ __global__ void exp2_check_kernel(const float* __restrict__ x, float* __restrict
 }  // namespace
 
 extern "C" {
+
+int ring_attn_wait_selftest(long long timeout_ns, ra_stream stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return RA_ERR_ARG;
+  int st = RA_OK;
+  if (!dev_info(&st)) return st;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(timeout_ns));
+  return launch_status();
+}
 
 int ring_attn_exp2_check(const float* x, float* y_fma, float* y_mufu, long long n, ra_stream stream) {
   if (!x || !y_fma || !y_mufu || n <= 0) return RA_ERR_ARG;

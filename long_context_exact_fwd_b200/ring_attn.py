@@ -50,6 +50,7 @@ _launch_count = _sig("ring_attn_launch_count", ctypes.c_ulonglong)
 _bwd_noalloc = _sig("ring_attn_bwd_noalloc", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _noalloc_max = _sig("ring_attn_bwd_noalloc_max_bytes", _sz)
 _exp2_check = _sig("ring_attn_exp2_check", _i, _vp, _vp, _vp, ctypes.c_longlong, _vp)
+_wait_selftest = _sig("ring_attn_wait_selftest", _i, ctypes.c_longlong, _vp)
 
 
 class RingAttnError(RuntimeError):
@@ -233,6 +234,11 @@ def exp2_check(x: torch.Tensor, stream=None):
     y1, y2 = torch.empty_like(x), torch.empty_like(x)
     _check(_exp2_check(x.data_ptr(), y1.data_ptr(), y2.data_ptr(), x.numel(), _stream(stream)), "ring_attn_exp2_check")
     return y1, y2
+
+
+def wait_selftest(timeout_s: float = 0.05, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (it records RA_ERR_TIMEOUT on purpose)."""
+    _check(_wait_selftest(int(timeout_s * 1e9), _stream(stream)), "ring_attn_wait_selftest")
 
 
 def launch_count() -> int:
