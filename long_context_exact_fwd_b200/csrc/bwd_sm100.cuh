@@ -65,8 +65,10 @@ static_assert(2 * (REGS_KEYS - REGS_LAUNCH) + (REGS_DQ - REGS_LAUNCH) <= REGS_LA
 static_assert(NUM_THREADS * REGS_LAUNCH <= 65536, "launch register budget");
 constexpr uint32_t TMEM_COLS = 512;
 // Of every 8 columns of P, 2 x this many exponentials run on the FMA pipes (exp2_fma2).
+// 0 by default: with four warpgroups the MUFU pipe keeps up, and moving exponentials to
+// the FMA pipes measured 8% slower at S = 16K, Dh = 128.
 #ifndef RA_BWD_EXP2_FMA_PER4
-#define RA_BWD_EXP2_FMA_PER4 1
+#define RA_BWD_EXP2_FMA_PER4 0
 #endif
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 384;
 // bf16 P^T / dS^T of query columns [64h, 64h + 64): TMEM columns [base, base + 32)

@@ -125,8 +125,11 @@ int check_shape(int B, int H, int S, int Dh, int D) {
 }
 
 // Heads whose per-head streamed operands (`bytes_per_head`) fit together in ~48 MiB of L2.
+#ifndef RA_L2_GROUP_MIB
+#define RA_L2_GROUP_MIB 48
+#endif
 int heads_per_l2_group(long long BH, long long bytes_per_head) {
-  const long long g = (48ll << 20) / (bytes_per_head > 0 ? bytes_per_head : 1);
+  const long long g = (static_cast<long long>(RA_L2_GROUP_MIB) << 20) / (bytes_per_head > 0 ? bytes_per_head : 1);
   return static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
 }
 
