@@ -21,6 +21,7 @@ algorithm against the plain definition.  No function here is "parity unpinned".
 """
 from .attention import (  # noqa: F401
     attn_fwd,
+    attn_fwd_keys,
     attn_fwd_heads,
     attn_bwd,
     attn_bwd_heads,

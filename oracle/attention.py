@@ -92,6 +92,36 @@ def attn_fwd(q, k, v, causal: bool, scale: Optional[float] = None,
     return O, L
 
 
+def attn_fwd_keys(q, k, v, keys: Sequence[int], causal: bool, scale: Optional[float] = None,
+                  rows: Optional[Sequence[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """One head, attention over the key positions ``keys`` only (global indices, any order):
+    for query row i the allowed set is {j in keys} (and j <= i when causal), and O_i, LSE_i
+    are attn_fwd's definition over that set; a row with no allowed key gets LSE = -inf and
+    O = 0.  This is one partial of "精读笔记 ..." §3.1: a query block against a subset of the
+    key/value blocks, to be combined with the others through lse_merge."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    S, Dh = q.shape
+    sc = _default_scale(Dh, scale)
+    idx = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    kk = np.asarray(keys, dtype=np.int64)
+    O = np.zeros((idx.size, v.shape[1]), dtype=np.float64)
+    L = np.full((idx.size,), NEG_INF, dtype=np.float64)
+    if kk.size == 0:
+        return O, L
+    s = (q[idx] @ k[kk].T) * sc
+    if causal:
+        s = np.where(kk[None, :] <= idx[:, None], s, NEG_INF)
+    m = s.max(axis=1)
+    ok = np.isfinite(m)
+    m_safe = np.where(ok, m, 0.0)
+    z = np.exp(s - m_safe[:, None]).sum(axis=1)
+    lse = np.where(ok, m_safe + np.log(np.where(ok, z, 1.0)), NEG_INF)
+    w = np.where(ok[:, None], np.exp(s - np.where(ok, lse, 0.0)[:, None]), 0.0)
+    O[:] = w @ v[kk]
+    L[:] = lse
+    return O, L
+
+
 def attn_fwd_heads(q, k, v, causal: bool, scale: Optional[float] = None,
                    rows=None, heads: Optional[Iterable[Tuple[int, int]]] = None
                    ) -> Tuple[np.ndarray, np.ndarray]:

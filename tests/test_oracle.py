@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from oracle import (attn_bwd, attn_fwd, attn_fwd_heads, lse_merge, ring_attention_blockwise,
+from oracle import (attn_bwd, attn_fwd, attn_fwd_heads, attn_fwd_keys, lse_merge, ring_attention_blockwise,
                     ring_attention_partials, ring_order)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -59,6 +59,60 @@ def test_fwd_matches_brute_force(causal, S, Dh):
     O, L = attn_fwd(q, k, v, causal)
     np.testing.assert_allclose(O, Ob, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(L, Lb, rtol=1e-12, atol=1e-12)
+
+
+def _brute_fwd_keys(q, k, v, keys, causal, scale):
+    """Scalar loops over an explicit key subset; global positions decide the mask."""
+    S, Dh, Dv = len(q), len(q[0]), len(v[0])
+    O, L = [], []
+    for i in range(S):
+        s = []
+        for j in keys:
+            if causal and j > i:
+                continue
+            s.append((j, sum(q[i][d] * k[j][d] for d in range(Dh)) * scale))
+        if not s:
+            O.append([0.0] * Dv)
+            L.append(-math.inf)
+            continue
+        M = max(x for _, x in s)
+        lse = M + math.log(sum(math.exp(x - M) for _, x in s))
+        o = [0.0] * Dv
+        for j, x in s:
+            for d in range(Dv):
+                o[d] += math.exp(x - lse) * v[j][d]
+        O.append(o)
+        L.append(lse)
+    return np.array(O), np.array(L)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_subset_matches_brute_force(causal):
+    S, Dh = 11, 4
+    q, k, v = (_rand((S, Dh), s) * 1.3 for s in (21, 22, 23))
+    keys = [9, 2, 5, 6]   # any order; rows 0 and 1 see none of them under the causal mask
+    Ob, Lb = _brute_fwd_keys(q.tolist(), k.tolist(), v.tolist(), keys, causal, 1.0 / math.sqrt(Dh))
+    O, L = attn_fwd_keys(q, k, v, keys, causal)
+    np.testing.assert_allclose(O, Ob, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(np.isinf(L), np.isinf(Lb))
+    fin = np.isfinite(Lb)
+    np.testing.assert_allclose(L[fin], Lb[fin], rtol=1e-12, atol=1e-12)
+    if causal:
+        assert np.isneginf(L[:2]).all() and not O[:2].any()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_partition_merges_to_full(causal):
+    # pieces of the key positions (one empty), merged through their lse, give the plain result
+    S, Dh = 50, 6
+    q, k, v = (_rand((S, Dh), s) for s in (31, 32, 33))
+    perm = np.random.default_rng(34).permutation(S)
+    pieces = [perm[:7], perm[7:7], perm[7:30], perm[30:]]
+    parts = [attn_fwd_keys(q, k, v, p, causal) for p in pieces]
+    O, L = lse_merge(np.stack([o for o, _ in parts]), np.stack([l for _, l in parts]))
+    Of, Lf = attn_fwd(q, k, v, causal)
+    np.testing.assert_allclose(O, Of, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(L, Lf, rtol=1e-12, atol=1e-12)
 
 
 def test_fwd_row_subset_and_chunking():
