@@ -238,7 +238,8 @@ def _config(w: Workload, args):
             "pass": "fwd+bwd" if w.backward else "fwd", "flops_per_step": w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0),
             "l2": ("working set %.0f MiB > %d MiB L2, not flushed" % (ws_bytes / 2 ** 20, L2_BYTES >> 20))
             if ws_bytes > 3 * L2_BYTES else "L2 flushed between steps (256 MiB write)",
-            "seeds": f"workload seed {w.seed} (+1000*rank)"}
+            "seeds": f"workload seed {w.seed} (+1000*rank)",
+            "fwd_parts": getattr(args, "parts", 1)}
 
 
 # ------------------------------------------------------------------------------- our arm
@@ -262,6 +263,10 @@ def run_ours(args, w: Workload):
     if w.backward:
         dq, dk, dv = (torch.empty_like(x["q"]) for _ in range(3))
         wsb = torch.empty(ra.bwd_workspace_bytes(w.B, w.H, w.S, w.Dh), dtype=torch.uint8, device=dev)
+    split_ws = None
+    if args.parts > 1:   # split-ring forward: pieces of each pair's ring merged through their lse
+        split_ws = torch.empty(ra.fwd_split_workspace_bytes(w.B, w.H, w.S, w.Dh, args.parts), dtype=torch.uint8,
+                               device=dev)
     stream = torch.cuda.current_stream(dev)
     flush_needed = "flushed" in _config(w, args)["l2"]
     flush_buf = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev) if flush_needed else None
@@ -269,7 +274,11 @@ def run_ours(args, w: Workload):
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        ra.fwd(x["q"], x["k"], x["v"], w.D, w.causal, out=o, lse=lse, stream=stream)
+        if split_ws is None:
+            ra.fwd(x["q"], x["k"], x["v"], w.D, w.causal, out=o, lse=lse, stream=stream)
+        else:
+            ra.fwd_split(x["q"], x["k"], x["v"], w.D, w.causal, n_parts=args.parts, workspace=split_ws,
+                         out=o, lse=lse, stream=stream)
         if evs:
             evs[1].record(stream)
         if w.backward:
@@ -362,7 +371,9 @@ def run_ours(args, w: Workload):
                 "peak_source": f"{src} {'sustained' if long_region else 'burst'} bf16 dense "
                                f"(MEASURED_PEAKS.json)" if src == "measured" else "fallback",
                 "timing": ("CUDA events around the %s call on its stream over the timed region" % dom)
-                + (" (includes its Delta preprocess and dQ convert kernels)" if dom == "ring_attn_bwd" else "")}
+                + (" (includes its Delta preprocess and dQ convert kernels)" if dom == "ring_attn_bwd" else "")
+                + (" (includes the merge of the %d pieces)" % args.parts if dom == "ring_attn_fwd" and args.parts > 1
+                   else "")}
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
             n = args.sample_rows or (w.S if w.backward else 2048)
@@ -392,6 +403,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[n for n in WORKLOADS if n != "tiny_fp32"])
     ap.add_argument("--sample-rows", type=int, default=0, help="oracle sample size (rows / causal prefix)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parts", type=int, default=1,
+                    help="forward: cut each query pair's ring into this many pieces (ring_attn_fwd_split)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # the timing rules ask for at least 3 warm-up steps
     w = WORKLOADS[args.workload]

@@ -52,7 +52,7 @@ enum {
   RA_ERR_ARG = 1,         /* null pointer, non-positive size, unknown dtype            */
   RA_ERR_SHAPE = 2,       /* S % D != 0, unsupported Dh, or a size that overflows       */
   RA_ERR_ALIGN = 3,       /* a TMA-read pointer is not 16-byte aligned                 */
-  RA_ERR_WORKSPACE = 4,   /* backward workspace null or smaller than required          */
+  RA_ERR_WORKSPACE = 4,   /* workspace null or smaller than required                   */
   RA_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed                      */
   RA_ERR_TIMEOUT = 6,     /* a kernel gave up on a bounded internal wait               */
   RA_ERR_DEVICE = 7       /* the current device is not compute capability 10.0         */
@@ -89,6 +89,42 @@ RA_API int ring_attn_fwd(const void* q, const void* k, const void* v, void* o, f
  */
 RA_API int ring_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
                      int Dh, int D, int causal, ra_dtype dtype, float scale, ra_stream stream);
+
+/* Largest n_parts ring_attn_fwd_split accepts. */
+#define RA_MAX_FWD_PARTS 16
+
+/*
+ * ring_attn_fwd_split_workspace_size -- bytes of device workspace ring_attn_fwd_split needs
+ * for n_parts pieces: n_parts float32 partial outputs [B][H][S][Dh] followed by n_parts
+ * float32 partial log-sum-exps [B][H][S] (that region rounded up to 256 bytes per part).
+ * Returns 0 for invalid sizes.
+ */
+RA_API size_t ring_attn_fwd_split_workspace_size(int B, int H, int S, int Dh, int n_parts);
+
+/*
+ * ring_attn_fwd_split -- forward pass with each query block's ring cut into pieces that run
+ * on different SMs, then merged (page "精读笔记 ...", §3.1: partial results over disjoint
+ * sets of key/value blocks, combined in any order through their statistics; page
+ * "RingAttention large-context attention", 架构与算法: partial outputs aggregated into the
+ * final output).  For few heads and long sequences the longest query blocks otherwise keep a
+ * handful of SMs busy after the rest have finished.
+ *   q, k, v, o, lse, B, H, S, Dh, D, causal  as ring_attn_fwd (Dh 64 or 128).
+ *   n_parts   1..RA_MAX_FWD_PARTS.  Each 256-row query pair's key tiles, in ring order, are
+ *             cut into n_parts contiguous pieces of near-equal tile count; piece p is one
+ *             work item.  A pair with fewer tiles than n_parts leaves some pieces empty
+ *             (lse -inf, weight 0 in the merge).  n_parts = 1 is ring_attn_fwd exactly and
+ *             needs no workspace.
+ *   workspace device memory of at least ring_attn_fwd_split_workspace_size(...) bytes,
+ *             256-byte aligned, owned by the caller; its contents on entry do not matter and
+ *             on return hold the partials (o_part, lse_part) for inspection.
+ * Two launches on `stream`: the forward kernel writing the partials, then ring_attn_merge.
+ * Errors: RA_ERR_ARG (null pointer, n_parts out of range), RA_ERR_SHAPE, RA_ERR_ALIGN (inputs
+ * not 16-byte or workspace not 256-byte aligned), RA_ERR_WORKSPACE (missing or too small),
+ * RA_ERR_CUDA.
+ */
+RA_API int ring_attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
+                               int Dh, int D, int causal, int n_parts, void* workspace, size_t workspace_bytes,
+                               ra_stream stream);
 
 /*
  * ring_attn_bwd_workspace_size -- bytes of device workspace ring_attn_bwd needs: a float32

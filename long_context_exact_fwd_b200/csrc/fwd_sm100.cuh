@@ -17,6 +17,9 @@
 // Issue order per key tile j (ping-pong, so the softmax of one query tile overlaps the
 // tensor-core work of the other):
 //   O0 += P0(j-1) V(j-1);  S0 = Q0 K(j)^T;  O1 += P1(j-1) V(j-1);  S1 = Q1 K(j)^T.
+// SPLIT = true (ring_attn_fwd_split): a work item is one piece of a pair's visit order
+// (RingTiles::restrict_to); the epilogue writes the piece's normalised fp32 O and its lse
+// for the merge instead of bf16 O.
 // Online softmax (base 2, scale folded in): the running max used as exponent reference is
 // only raised when the tile max exceeds it by more than 8 (a factor 256), so O is rescaled
 // in TMEM rarely; any reference gives the same O / l exactly in real arithmetic.
@@ -78,25 +81,33 @@ struct Layout {
 struct Params {
   int BH, S, D, causal;
   int n_pairs;        // ceil(S / ROWS)
-  int n_items;        // BH * n_pairs
+  int n_parts;        // pieces each pair's visit order is cut into (1: no split)
+  int n_items;        // BH * n_pairs * n_parts
   int hgroup;         // heads whose items are interleaved (L2 reuse of K, V)
   int work_slot;      // this launch's work counter
   float scale_log2;   // softmax scale * log2(e)
-  __nv_bfloat16* o;   // [BH][S][HD]
+  __nv_bfloat16* o;   // [BH][S][HD]                  (n_parts == 1)
   float* lse;         // [BH][S]
+  float* o_part;      // [n_parts][BH][S][HD] fp32, normalised per part   (n_parts > 1)
+  float* lse_part;    // [n_parts][BH][S], natural log, -inf for a row that sees no key of the part
 };
 
-// Work item w -> (bh, pair).  Heads are taken in groups of p.hgroup (all heads by default);
-// inside a group items go pair by pair, causal: the last query tiles (longest items) first,
-// so the CTAs that fetch items dynamically finish together.
-__device__ __forceinline__ void item_coords(int w, const Params& p, int& bh, int& pair) {
-  const int per_group = p.hgroup * p.n_pairs;
+// Work item w -> (bh, pair, part).  Heads are taken in groups of p.hgroup (all heads by
+// default); inside a group items go pair by pair, causal: the last query tiles (longest
+// items) first, so the CTAs that fetch items dynamically finish together; the parts of one
+// pair are adjacent.
+template <bool SPLIT>
+__device__ __forceinline__ void item_coords(int w, const Params& p, int& bh, int& pair, int& part) {
+  const int n_parts = SPLIT ? p.n_parts : 1;
+  const int per_group = p.hgroup * p.n_pairs * n_parts;
   const int g = w / per_group;
   const int gsize = min(p.hgroup, p.BH - g * p.hgroup);
   const int idx = w - g * per_group;
   const int rank = idx / gsize;
   bh = g * p.hgroup + (idx - rank * gsize);
-  pair = p.causal ? (p.n_pairs - 1 - rank) : rank;
+  const int pair_rank = SPLIT ? rank / n_parts : rank;
+  part = rank - pair_rank * n_parts;
+  pair = p.causal ? (p.n_pairs - 1 - pair_rank) : pair_rank;
 }
 
 __device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
@@ -107,7 +118,7 @@ __device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
 }
 
 // ------------------------------------------------------------------ producer (1 thread)
-template <int HD>
+template <int HD, bool SPLIT>
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const Params& p, uint32_t sbase, volatile int* wq, volatile int* abort_flag) {
   using L = Layout<HD>;
@@ -125,9 +136,15 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
     if (!ring.push(w, abort_flag)) { ok = false; break; }
     if (w >= p.n_items) break;
     const int w_next = work_fetch(p.work_slot);   // in flight while this item's loads issue
-    int bh, pair;
-    item_coords(w, p, bh, pair);
+    int bh, pair, part;
+    item_coords<SPLIT>(w, p, bh, pair, part);
     const int q0 = pair * ROWS;
+    RingTiles it;
+    it.init(p.S, p.D, p.causal, q0, ROWS, BN);
+    if (SPLIT && it.restrict_to(part, p.n_parts) == 0) {   // empty piece: nothing to load
+      w = w_next;
+      continue;
+    }
     if (!mbar_wait(bar(L::B_Q_EMPTY), q_phase ^ 1u, abort_flag)) { ok = false; break; }
     mbar_arrive_expect_tx(bar(L::B_Q_FULL), NQ * L::TILE_BYTES);
 #pragma unroll
@@ -140,9 +157,7 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
     q_parity = q_phase;
     q_phase ^= 1u;
 
-    RingTiles it;
-    it.init(p.S, p.D, p.causal, q0, ROWS, BN);
-    for (int kt = it.next(); kt >= 0; kt = it.next()) {
+    for (int kt = (SPLIT ? it.next_in_part() : it.next()); kt >= 0; kt = (SPLIT ? it.next_in_part() : it.next())) {
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         if (!mbar_wait(bar(L::B_KV_EMPTY + stage), phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -198,7 +213,7 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, i
   }
 }
 
-template <int HD>
+template <int HD, bool SPLIT>
 __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
   using L = Layout<HD>;
   const uint32_t bars = sbase + L::BAR_OFF;
@@ -212,15 +227,16 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
     int w;
     if (!ring.pop(w, abort_flag)) { ok = false; break; }
     if (w >= p.n_items) break;
-    int bh, pair;
-    item_coords(w, p, bh, pair);
+    int bh, pair, part;
+    item_coords<SPLIT>(w, p, bh, pair, part);
+    RingTiles it;
+    it.init(p.S, p.D, p.causal, pair * ROWS, ROWS, BN);
+    if (SPLIT && it.restrict_to(part, p.n_parts) == 0) continue;   // empty piece
     if (!mbar_wait(bar(L::B_Q_FULL), q_phase, abort_flag)) { ok = false; break; }
     q_phase ^= 1u;
     tc_fence_after();
-    RingTiles it;
-    it.init(p.S, p.D, p.causal, pair * ROWS, ROWS, BN);
     int vprev = 0, n = 0;
-    for (int kt = it.next(); kt >= 0; kt = it.next(), ++n) {
+    for (int kt = (SPLIT ? it.next_in_part() : it.next()); kt >= 0; kt = (SPLIT ? it.next_in_part() : it.next()), ++n) {
       const int ks = stage;
       if (!mbar_wait(bar(L::B_KV_FULL + ks), phase, abort_flag)) { ok = false; break; }
       advance(stage, phase);
@@ -264,7 +280,7 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
 }
 
 // ------------------------------------------------------------------ softmax (128 threads)
-template <int HD>
+template <int HD, bool SPLIT>
 __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq,
                            volatile int* abort_flag) {
   using L = Layout<HD>;
@@ -284,17 +300,28 @@ __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem
     int w;
     if (!ring.pop_warp(w, abort_flag)) return;
     if (w >= p.n_items) break;
-    int bh, pair;
-    item_coords(w, p, bh, pair);
+    int bh, pair, part;
+    item_coords<SPLIT>(w, p, bh, pair, part);
     const int q_tile0 = pair * ROWS + t * BM;
     const int q_row = q_tile0 + row;
     const int vis_end = (p.causal && q_row + 1 < p.S) ? q_row + 1 : p.S;  // keys [0, vis_end) visible
+    const bool row_ok = q_row < p.S;
     float m_ref = -INFINITY;   // exponent reference (log2 units), raised lazily
     float l = 0.f;
     RingTiles it;
     it.init(p.S, p.D, p.causal, pair * ROWS, ROWS, BN);
+    if (SPLIT && it.restrict_to(part, p.n_parts) == 0) {   // empty piece: O = 0, lse = -inf
+      if (row_ok) {
+        const size_t prow = (static_cast<size_t>(part) * p.BH + bh) * p.S + q_row;
+        float4* dst = reinterpret_cast<float4*>(p.o_part + prow * HD);
+#pragma unroll
+        for (int i = 0; i < HD / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        p.lse_part[prow] = -INFINITY;
+      }
+      continue;
+    }
     int n = 0;
-    for (int kt = it.next(); kt >= 0; kt = it.next(), ++n) {
+    for (int kt = (SPLIT ? it.next_in_part() : it.next()); kt >= 0; kt = (SPLIT ? it.next_in_part() : it.next()), ++n) {
       // all 32 lanes must agree before the warp-collective TMEM loads below
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_S_FULL + t), s_phase, abort_flag))) return;
       s_phase ^= 1u;
@@ -378,7 +405,26 @@ __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem
     o_phase ^= 1u;
     tc_fence_after();
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    const bool row_ok = q_row < p.S;
+    const float lse_row = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (SPLIT) {   // normalised fp32 partial of this piece, merged through its lse
+      const size_t prow = (static_cast<size_t>(part) * p.BH + bh) * p.S + q_row;
+      float* orow = p.o_part + prow * HD;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_ld_wait();
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                 __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+        }
+      }
+      if (row_ok) p.lse_part[prow] = lse_row;
+      continue;
+    }
     __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.S + q_row) * HD;
 #pragma unroll
     for (int c = 0; c < HD / 32; ++c) {
@@ -395,14 +441,12 @@ __device__ void softmax_wg(int t, const Params& p, uint32_t sbase, uint32_t tmem
         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w16[4 * i], w16[4 * i + 1], w16[4 * i + 2], w16[4 * i + 3]);
       }
     }
-    if (row_ok)
-      p.lse[static_cast<size_t>(bh) * p.S + q_row] =
-          l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (row_ok) p.lse[static_cast<size_t>(bh) * p.S + q_row] = lse_row;
   }
 }
 
 // ------------------------------------------------------------------ kernel
-template <int HD>
+template <int HD, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -442,15 +486,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp >= 8) {
     regs_lower<REGS_OTHER>();
     if (warp == WARP_TMA) {
-      if ((threadIdx.x & 31) == 0) producer<HD>(&tm_q, &tm_k, &tm_v, p, sbase, wq, abort_flag);
+      if ((threadIdx.x & 31) == 0) producer<HD, SPLIT>(&tm_q, &tm_k, &tm_v, p, sbase, wq, abort_flag);
       __syncwarp();
     } else if (warp == WARP_MMA) {
-      if ((threadIdx.x & 31) == 0) mma_issuer<HD>(p, sbase, tmem, wq, abort_flag);
+      if ((threadIdx.x & 31) == 0) mma_issuer<HD, SPLIT>(p, sbase, tmem, wq, abort_flag);
       __syncwarp();
     }
   } else {
     regs_raise<REGS_SOFTMAX>();
-    softmax_wg<HD>(warp >> 2, p, sbase, tmem, wq, abort_flag);
+    softmax_wg<HD, SPLIT>(warp >> 2, p, sbase, tmem, wq, abort_flag);
   }
 
   tc_fence_before();

@@ -54,6 +54,41 @@ struct RingTiles {
     }
     return -1;
   }
+
+  // Number of key tiles the whole visit order holds (call right after init; leaves the
+  // iterator where init put it).
+  RA_HD int count() const {
+    int n = 0;
+    for (int u = 0; u < D; ++u) {
+      const int j = ((r - u) % D + D) % D;
+      const int a = cdiv(static_cast<long long>(j) * c, kt_size);
+      const int e0 = cdiv(static_cast<long long>(j + 1) * c, kt_size);
+      const int e = e0 < kt_limit ? e0 : kt_limit;
+      if (e > a) n += e - a;
+    }
+    return n;
+  }
+
+  // Restrict the iterator to part `part` of `n_parts` contiguous, near-equal pieces of the
+  // visit order (pieces [n*part/n_parts, n*(part+1)/n_parts) of the n tiles); returns the
+  // number of tiles in the piece (0 when n < n_parts leaves it empty).  Call right after init.
+  RA_HD int restrict_to(int part, int n_parts) {
+    const int n = count();
+    const int lo = static_cast<int>(static_cast<long long>(n) * part / n_parts);
+    const int hi = static_cast<int>(static_cast<long long>(n) * (part + 1) / n_parts);
+    for (int i = 0; i < lo; ++i) next();
+    left = hi - lo;
+    return left;
+  }
+
+  // next() bounded by restrict_to's piece (call instead of next() after restrict_to).
+  RA_HD int next_in_part() {
+    if (left <= 0) return -1;
+    --left;
+    return next();
+  }
+
+  int left = 1 << 30;   // tiles next_in_part may still return (unbounded until restrict_to)
 };
 
 // The backward's view of the same ring: key/value block j sits at ring position

@@ -56,7 +56,7 @@ struct DevInfo {
   int sm_count = 0;
   std::atomic<unsigned> next_work_slot{0};   // round robin over the kernels' work counters
   bool ok = false;          // compute capability 10.0
-  bool fwd_attr[2] = {false, false};
+  bool fwd_attr[4] = {false, false, false, false};   // [HD 128, HD 64] x [whole ring, split]
   bool bwd_attr = false;
 };
 
@@ -139,9 +139,11 @@ int launch_status() {
   return e == cudaSuccess ? RA_OK : cuda_fail(static_cast<int>(e), "kernel launch");
 }
 
+// n_parts > 1: each query pair's visit order is cut into n_parts pieces, written as fp32
+// partials to o_part / lse_part ([n_parts][B*H][S][HD], [n_parts][B*H][S]) for the merge.
 template <int HD>
 int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D, int causal,
-             float scale, cudaStream_t stream) {
+             float scale, cudaStream_t stream, int n_parts = 1, float* o_part = nullptr, float* lse_part = nullptr) {
   using namespace ra::fwd;
   int st = RA_OK;
   DevInfo* di = dev_info(&st);
@@ -157,7 +159,8 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.D = D;
   p.causal = causal ? 1 : 0;
   p.n_pairs = (S + ROWS - 1) / ROWS;
-  const long long items = BH * p.n_pairs;
+  p.n_parts = n_parts;
+  const long long items = BH * p.n_pairs * n_parts;
   if (items > INT_MAX) return RA_ERR_SHAPE;
   p.n_items = static_cast<int>(items);
   // All heads interleaved: with dynamic scheduling this measured best per cycle at S = 16K
@@ -167,15 +170,19 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
   constexpr int smem = Layout<HD>::ALLOC;
-  const int slot = HD == 128 ? 0 : 1;
+  const bool split = n_parts > 1;
+  const int slot = (HD == 128 ? 0 : 1) + (split ? 2 : 0);
+  auto kern = split ? fwd_kernel<HD, true> : fwd_kernel<HD, false>;
   if (!di->fwd_attr[slot]) {
-    const cudaError_t e = cudaFuncSetAttribute(fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(fwd smem)");
     di->fwd_attr[slot] = true;
   }
   const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
-  fwd_kernel<HD><<<grid, NUM_THREADS, smem, stream>>>(mq, mk, mv, p);
+  kern<<<grid, NUM_THREADS, smem, stream>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -374,6 +381,42 @@ int ring_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float
 int ring_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int Dh, int D,
                   int causal, ra_stream stream) {
   return ring_attn_fwd_ex(q, k, v, o, lse, B, H, S, Dh, D, causal, RA_BF16, 0.f, stream);
+}
+
+size_t ring_attn_fwd_split_workspace_size(int B, int H, int S, int Dh, int n_parts) {
+  if (B <= 0 || H <= 0 || S <= 0 || Dh <= 0 || n_parts <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * S;
+  // fp32 partial O, then the partial lse, each part's block 256-B aligned
+  const size_t o_bytes = (rows * Dh * 4 + 255) / 256 * 256;
+  const size_t l_bytes = (rows * 4 + 255) / 256 * 256;
+  return static_cast<size_t>(n_parts) * (o_bytes + l_bytes);
+}
+
+int ring_attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int Dh,
+                        int D, int causal, int n_parts, void* workspace, size_t workspace_bytes, ra_stream stream) {
+  if (!q || !k || !v || !o || !lse) return RA_ERR_ARG;
+  if (n_parts <= 0 || n_parts > RA_MAX_FWD_PARTS) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  if (Dh != 128 && Dh != 64) return RA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RA_ERR_ALIGN;
+  const float sc = 1.f / std::sqrt(static_cast<float>(Dh));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_parts == 1) return Dh == 128 ? fwd_bf16<128>(q, k, v, o, lse, B, H, S, D, causal, sc, s)
+                                     : fwd_bf16<64>(q, k, v, o, lse, B, H, S, D, causal, sc, s);
+  const size_t need = ring_attn_fwd_split_workspace_size(B, H, S, Dh, n_parts);
+  if (!workspace || workspace_bytes < need) return RA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return RA_ERR_ALIGN;
+  const size_t rows = static_cast<size_t>(B) * H * S;
+  const size_t o_bytes = (rows * Dh * 4 + 255) / 256 * 256;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + static_cast<size_t>(n_parts) * o_bytes);
+  // the merge reads part p at o_part + p * rows * Dh: keep the parts densely packed
+  if (o_bytes != rows * Dh * 4) return RA_ERR_SHAPE;
+  st = Dh == 128 ? fwd_bf16<128>(q, k, v, o, lse, B, H, S, D, causal, sc, s, n_parts, o_part, lse_part)
+                 : fwd_bf16<64>(q, k, v, o, lse, B, H, S, D, causal, sc, s, n_parts, o_part, lse_part);
+  if (st != RA_OK) return st;
+  return ring_attn_merge(o_part, lse_part, n_parts, o, lse, B, H, S, Dh, stream);
 }
 
 int ring_attn_merge_ex(const float* o_parts, const float* lse_parts, int P, void* o, float* lse, int B, int H, int S,

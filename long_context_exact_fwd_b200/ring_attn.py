@@ -37,6 +37,8 @@ def _sig(name, restype, *argtypes):
 _fwd = _sig("ring_attn_fwd", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _fwd_ex = _sig("ring_attn_fwd_ex", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp)
 _bwd_ws = _sig("ring_attn_bwd_workspace_size", _sz, _i, _i, _i, _i)
+_split_ws = _sig("ring_attn_fwd_split_workspace_size", _sz, _i, _i, _i, _i, _i)
+_fwd_split = _sig("ring_attn_fwd_split", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
 _bwd = _sig("ring_attn_bwd", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
 _merge_ex = _sig("ring_attn_merge_ex", _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp)
 _ring_order = _sig("ring_attn_ring_order", _i, _i, _i, _i, _ip, _i)
@@ -126,6 +128,50 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, D: int, causal: bool 
                    1 if causal else 0, RA_BF16 if dt == torch.bfloat16 else RA_F32,
                    float(scale) if scale else 0.0, _stream(stream))
     _check(code, "ring_attn_fwd")
+    return out, lse
+
+
+def fwd_split_workspace_bytes(B: int, H: int, S: int, Dh: int, n_parts: int) -> int:
+    return int(_split_ws(B, H, S, Dh, n_parts))
+
+
+def split_parts_hint(B: int, H: int, S: int, device=None) -> int:
+    """Pieces per query pair worth using: 2 while the forward has fewer than two 256-row work
+    items per SM (measured on B200: H=1 S=64K +50 %, H=2 S=32K +31 %; from four items per SM
+    on, splitting only adds the merge), else 1."""
+    sms = torch.cuda.get_device_properties(device if device is not None else torch.cuda.current_device()) \
+        .multi_processor_count
+    items = B * H * ((S + 255) // 256)
+    return 2 if items < 2 * sms else 1
+
+
+def fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, D: int, causal: bool = True,
+              n_parts: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+              stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Forward with each query pair's ring cut into n_parts pieces merged through their
+    log-sum-exp (ring_attn_fwd_split); n_parts None picks split_parts_hint.  q, k, v:
+    [B, H, S, Dh] bf16.  Returns (o, lse); after the call `workspace` (if given) holds the
+    partials."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, S, Dh]")
+    B, H, S, Dh = q.shape
+    if n_parts is None:
+        n_parts = split_parts_hint(B, H, S, q.device)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, q.shape)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(out, "out", torch.bfloat16, q.shape)
+    _need(lse, "lse", torch.float32, (B, H, S))
+    need = fwd_split_workspace_bytes(B, H, S, Dh, n_parts)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    code = _fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, S, Dh, D,
+                      1 if causal else 0, n_parts, workspace.data_ptr(),
+                      workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "ring_attn_fwd_split")
     return out, lse
 
 

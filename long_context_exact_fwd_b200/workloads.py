@@ -84,6 +84,9 @@ WORKLOADS: Dict[str, Workload] = {
                  sample_rows=128),
         Workload("s16k_fwd_bwd", B=1, H=16, S=16384, Dh=128, D=8, dtype="bf16", causal=True,
                  seed=4, backward=True, oracle_heads=(0, 15)),
+        Workload("s32k_h2", B=1, H=2, S=32768, Dh=128, D=8, dtype="bf16", causal=True, seed=5,
+                 sample_rows=256,
+                 note="few heads, long rows: 256 query-pair items for 148 SMs (split-ring case)"),
     )
 }
 

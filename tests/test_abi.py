@@ -75,6 +75,27 @@ def test_merge_and_bwd_argument_errors(ra):
     assert ra.bwd_workspace_bytes(0, 2, 256, 128) == 0
 
 
+def test_split_forward_workspace_and_argument_errors(ra):
+    rows = 1 * 2 * 1000
+    lse_block = (rows * 4 + 255) // 256 * 256
+    assert ra.fwd_split_workspace_bytes(1, 2, 1000, 128, 3) == 3 * rows * 128 * 4 + 3 * lse_block
+    assert ra.fwd_split_workspace_bytes(1, 2, 1000, 128, 0) == 0
+    f = ra.raw.ring_attn_fwd_split
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    args = lambda **kw: [P(kw.get("q", 256)), P(256), P(256), P(256), P(256), 1, 2, 1024, 128, 4, 1,
+                         kw.get("n_parts", 2), P(kw.get("ws", 256)), ctypes.c_size_t(kw.get("ws_bytes", 1 << 40)),
+                         P(0)]
+    # all rejected before anything is enqueued (no device needed)
+    assert f(*args(q=0)) == ra.RA_ERR_ARG
+    assert f(*args(n_parts=0)) == ra.RA_ERR_ARG
+    assert f(*args(n_parts=17)) == ra.RA_ERR_ARG
+    assert f(*args(ws=0)) == ra.RA_ERR_WORKSPACE
+    assert f(*args(ws_bytes=1024)) == ra.RA_ERR_WORKSPACE
+    assert f(*args(ws=272)) == ra.RA_ERR_ALIGN          # workspace must be 256-byte aligned
+    assert f(*args(q=24)) == ra.RA_ERR_ALIGN
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_library_ring_order_matches_oracle(ra, causal):
     for D in (1, 2, 3, 4, 7, 8, 16):
