@@ -24,6 +24,7 @@ from .attention import (  # noqa: F401
     attn_fwd_keys,
     attn_fwd_heads,
     attn_bwd,
+    attn_bwd_given_stats,
     attn_bwd_heads,
     lse_merge,
     ring_order,

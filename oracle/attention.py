@@ -176,6 +176,29 @@ def attn_bwd(q, k, v, do, causal: bool, scale: Optional[float] = None, chunk: in
     return dq, dk, dv
 
 
+def attn_bwd_given_stats(q, k, v, o, lse, do, causal: bool, scale: Optional[float] = None
+                         ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """One head, one query block against one key/value block, with the row statistics O and
+    LSE of the full rows (every key block): P = exp(S - LSE), dV = P^T dO, dP = dO V^T,
+    Delta = rowsum(dO * O), dS = P * (dP - Delta), dQ = scale dS K, dK = scale dS^T Q.
+    ``causal`` masks key i > query i inside the pair (the diagonal block, same positions).
+    Summing dQ over a row's key blocks, and dK, dV over a key block's query blocks, gives
+    attn_bwd -- the ring backward's per-step contribution."""
+    q, k, v, o, do = _as64(q), _as64(k), _as64(v), _as64(o), _as64(do)
+    lse = np.asarray(lse, dtype=np.float64)
+    sc = _default_scale(q.shape[1], scale)
+    s = (q @ k.T) * sc
+    if causal:
+        n, m = s.shape
+        s = np.where(np.arange(m)[None, :] <= np.arange(n)[:, None], s, NEG_INF)
+    p = np.exp(s - lse[:, None])
+    dv = p.T @ do
+    dp = do @ v.T
+    delta = (do * o).sum(axis=1)
+    ds = p * (dp - delta[:, None])
+    return sc * (ds @ k), sc * (ds.T @ q), dv
+
+
 def attn_bwd_heads(q, k, v, do, causal: bool, scale: Optional[float] = None,
                    heads: Optional[Iterable[Tuple[int, int]]] = None):
     """[B, H, S, Dh] inputs; gradients for the listed (b, h) heads (others NaN)."""

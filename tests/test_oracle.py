@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from oracle import (attn_bwd, attn_fwd, attn_fwd_heads, attn_fwd_keys, lse_merge, ring_attention_blockwise,
+from oracle import (attn_bwd, attn_bwd_given_stats, attn_fwd, attn_fwd_heads, attn_fwd_keys, lse_merge, ring_attention_blockwise,
                     ring_attention_partials, ring_order)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -113,6 +113,31 @@ def test_key_partition_merges_to_full(causal):
     Of, Lf = attn_fwd(q, k, v, causal)
     np.testing.assert_allclose(O, Of, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(L, Lf, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_gradients_with_full_row_statistics_sum_to_the_gradient(causal):
+    # two blocks of c positions; per-pair gradients with the full rows' O and LSE, summed over
+    # the pairs a block takes part in, reproduce attn_bwd (whose own forward is the plain one)
+    c, Dh = 9, 5
+    q, k, v, do = (_rand((2 * c, Dh), s) for s in (41, 42, 43, 44))
+    O, L = attn_fwd(q, k, v, causal)
+    dQ, dK, dV = attn_bwd(q, k, v, do, causal)
+    blk = [slice(0, c), slice(c, 2 * c)]
+    dq = [np.zeros((c, Dh)) for _ in blk]
+    dk = [np.zeros((c, Dh)) for _ in blk]
+    dv = [np.zeros((c, Dh)) for _ in blk]
+    for r, qs in enumerate(blk):
+        for j, ks in enumerate(blk):
+            if causal and j > r:
+                continue
+            a, b, e = attn_bwd_given_stats(q[qs], k[ks], v[ks], O[qs], L[qs], do[qs], causal and j == r)
+            dq[r] += a
+            dk[j] += b
+            dv[j] += e
+    np.testing.assert_allclose(np.concatenate(dq), dQ, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(dk), dK, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(dv), dV, rtol=1e-11, atol=1e-12)
 
 
 def test_fwd_row_subset_and_chunking():
