@@ -1,0 +1,104 @@
+"""Sequence-sharded ring (ring_dist.ring_fwd / ring_bwd) on CPU: 2 and 4 gloo ranks.
+
+Each rank holds one block of the sequence and the key/value blocks travel around the ring
+("精读笔记 ..." §3.2-§3.5).  The per-block work is injected here as the float64 oracle (the
+product binds the CUDA library instead), so these tests check the orchestration -- ring order,
+causal block skipping, neighbour send/receive pairing, the LSE merge, and the travelling dK/dV
+accumulators -- against the oracle's full-sequence attention and gradient.  No GPU.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _per_head(fn, *xs):
+    B, H = xs[0].shape[:2]
+    outs = None
+    for b in range(B):
+        for h in range(H):
+            res = fn(*[x[b, h].numpy() if isinstance(x, torch.Tensor) else x for x in xs])
+            if outs is None:
+                outs = [np.zeros((B, H) + np.shape(r)) for r in res]
+            for o, r in zip(outs, res):
+                o[b, h] = r
+    return [torch.from_numpy(o) for o in outs]
+
+
+def _full_inputs(B, H, S, Dh, seed):
+    g = torch.Generator().manual_seed(seed)
+    return [torch.randn(B, H, S, Dh, generator=g, dtype=torch.float64) for _ in range(4)]
+
+
+def _rank_main(rank, world, port, causal, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import oracle
+    from long_context_exact_fwd_b200 import ring_dist
+
+    def block_fwd(q, k, v, masked):
+        return _per_head(lambda a, b, c: oracle.attn_fwd(a, b, c, masked), q, k, v)
+
+    def merge(o_parts, lse_parts):
+        o, l = oracle.lse_merge(o_parts.numpy(), lse_parts.numpy())
+        return torch.from_numpy(o), torch.from_numpy(l)
+
+    def block_bwd(q, k, v, o, lse, do, masked):
+        return _per_head(lambda a, b, c, d, e, f: oracle.attn_bwd_given_stats(a, b, c, d, e, f, masked),
+                         q, k, v, o, lse, do)
+
+    B, H, c, Dh = 1, 2, 6, 4
+    q, k, v, do = _full_inputs(B, H, world * c, Dh, seed=11)
+    blk = slice(rank * c, (rank + 1) * c)
+    o, lse = ring_dist.ring_fwd(q[:, :, blk].contiguous(), k[:, :, blk].contiguous(), v[:, :, blk].contiguous(),
+                                causal, block_fwd=block_fwd, merge=merge)
+    dq, dk, dv = ring_dist.ring_bwd(q[:, :, blk].contiguous(), k[:, :, blk].contiguous(), v[:, :, blk].contiguous(),
+                                    o, lse, do[:, :, blk].contiguous(), causal, block_bwd=block_bwd)
+    O, L = _per_head(lambda a, b, cc: oracle.attn_fwd(a, b, cc, causal), q, k, v)
+    dQ, dK, dV = _per_head(lambda a, b, cc, d: oracle.attn_bwd(a, b, cc, d, causal), q, k, v, do)
+    err = lambda x, y: float((x.double() - y[:, :, blk]).abs().max())
+    out[rank] = (err(o, O), err(lse, L), err(dq, dQ), err(dk, dK), err(dv, dV))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_over_gloo_ranks_matches_the_full_oracle(world, causal):
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(world, _free_port(), causal, out), nprocs=world, join=True)
+        res = dict(out)
+    assert sorted(res) == list(range(world))
+    for rank, errs in res.items():
+        # the ring accumulates float32 partials of float64 blocks
+        assert max(errs) < 1e-5, (rank, errs)
+
+
+def test_ring_steps_follow_the_pages_ring_order():
+    sys.path.insert(0, ROOT)
+    import oracle
+    from long_context_exact_fwd_b200.ring_dist import ring_steps
+    for world in (1, 2, 4, 7):
+        for rank in range(world):
+            for causal in (False, True):
+                steps = ring_steps(rank, world, causal)
+                assert [j for _, j, _ in steps] == oracle.ring_order(world, rank, causal)
+                assert [m for _, j, m in steps] == [causal and j == rank for _, j, _ in steps]
+                assert steps[0][:2] == (0, rank)   # own block first

@@ -1,0 +1,68 @@
+"""The sequence-sharded ring's block-pair work on one B200, through the CUDA library.
+
+ring_dist.ring_fwd_emulated / ring_bwd_emulated run every rank of a D-rank ring in one process
+with the same ring_steps schedule as the distributed ring_fwd / ring_bwd (no communication: the
+blocks come from lists), so each block pair goes through ring_attn_fwd / ring_attn_bwd with the
+mask the ring gives it, and the partials through ring_attn_merge.  Compared with the float64
+oracle over the whole sequence.
+
+Forward bar: the bf16 parity bar (max-abs 2e-2, mean-abs 2e-3, LSE 1e-3).  Backward: each of a
+row's up to D per-step contributions comes back from the library rounded to bf16 and is summed
+in float32, so the bound is (D + 1) half-ulps of bf16 at the largest reference value, with the
+usual mean-abs 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_exact_fwd_b200.workloads import random_qkv
+from parity import assert_close_bf16, assert_lse
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rd():
+    from long_context_exact_fwd_b200 import build
+    build.ensure_built()
+    from long_context_exact_fwd_b200 import ring_dist
+    return ring_dist
+
+
+def _blocks(x, D):
+    return [b.contiguous() for b in x.chunk(D, dim=2)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D,c", [(2, 384), (4, 256)])
+def test_emulated_ring_forward_and_backward(rd, causal, D, c):
+    inp = random_qkv(1, 2, D * c, 128, seed=61 + D, with_do=True)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    outs = rd.ring_fwd_emulated(_blocks(q, D), _blocks(k, D), _blocks(v, D), causal)
+    o = torch.cat([x for x, _ in outs], dim=2)
+    lse = torch.cat([l for _, l in outs], dim=2)
+    O, L = oracle.attn_fwd_heads(inp["q"], inp["k"], inp["v"], causal)
+    assert_close_bf16(o.float().cpu().numpy(), O, "ring o")
+    assert_lse(lse.cpu().numpy(), L)
+
+    dq, dk, dv = rd.ring_bwd_emulated(_blocks(q, D), _blocks(k, D), _blocks(v, D), _blocks(o, D), _blocks(lse, D),
+                                      _blocks(do, D), causal)
+    ref = oracle.attn_bwd_heads(inp["q"], inp["k"], inp["v"], inp["do"], causal)
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        g = torch.cat(got, dim=2).float().cpu().numpy()
+        bound = (D + 1) * 2.0 ** -9 * np.abs(want).max()
+        err = np.abs(g - want)
+        assert err.max() <= max(bound, 2e-2), (name, err.max(), bound)
+        assert err.mean() <= 2e-3, (name, err.mean())
+
+
+def test_one_rank_ring_is_the_plain_forward(rd):
+    # no process group: a ring of one rank, one block, one merge of a single part
+    from long_context_exact_fwd_b200 import ring_attn as ra
+    inp = random_qkv(1, 2, 640, 128, seed=3)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o1, l1 = rd.ring_fwd(q, k, v, True)
+    o2, l2 = ra.fwd(q, k, v, 1, True)
+    assert torch.equal(o1, o2)
+    assert torch.allclose(l1, l2, atol=1e-6, rtol=0)
