@@ -49,7 +49,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_rank_gloo_group_max_time_and_job_throughput():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)

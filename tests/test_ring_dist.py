@@ -81,7 +81,7 @@ def _rank_main(rank, world, port, causal, out):
 @pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("causal", [False, True])
 def test_ring_over_gloo_ranks_matches_the_full_oracle(world, causal):
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), causal, out), nprocs=world, join=True)
         res = dict(out)
