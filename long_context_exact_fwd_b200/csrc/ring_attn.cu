@@ -429,9 +429,12 @@ int ring_attn_merge_ex(const float* o_parts, const float* lse_parts, int P, void
   const long long rows = static_cast<long long>(B) * H * S;
   if (static_cast<double>(rows) * P * Dh > 9.0e18 / 4) return RA_ERR_SHAPE;
   int st = RA_OK;
-  if (!dev_info(&st)) return st;
-  const long long blocks = (rows + ra::merge::WARPS - 1) / ra::merge::WARPS;
-  if (blocks > INT_MAX) return RA_ERR_SHAPE;
+  DevInfo* di = dev_info(&st);
+  if (!di) return st;
+  // persistent grid: a full SM's worth of blocks per SM, striding over the rows
+  long long blocks = (rows + ra::merge::WARPS - 1) / ra::merge::WARPS;
+  const long long cap = static_cast<long long>(di->sm_count) * ra::merge::BLOCKS_PER_SM;
+  if (blocks > cap) blocks = cap;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (out_dtype == RA_BF16)
     ra::merge::merge_kernel<__nv_bfloat16><<<static_cast<int>(blocks), ra::merge::WARPS * 32, 0, s>>>(

@@ -176,6 +176,25 @@ def test_merge_matches_oracle(ra, out_dtype):
     assert np.isneginf(lse[1, 2, 7].item()) and torch.all(o[1, 2, 7] == 0)
 
 
+@pytest.mark.parametrize("P,Dh", [(1, 128), (4, 64), (9, 256), (3, 36)])
+def test_merge_part_counts_head_dims_and_ignored_parts(ra, P, Dh):
+    # chunks of four partials with remainders, Dh not a multiple of 128, and partials marked
+    # -inf whose O holds NaN: they weigh 0 and must not reach the result
+    g = torch.Generator().manual_seed(20 + P)
+    B, H, S = 1, 2, 77
+    o_parts = torch.randn((P, B, H, S, Dh), generator=g)
+    lse_parts = torch.randn((P, B, H, S), generator=g) * 3
+    if P > 1:
+        lse_parts[P - 1, 0, 1, ::3] = float("-inf")
+        o_parts[P - 1, 0, 1, ::3] = float("nan")
+    o, lse = ra.merge(o_parts.cuda(), lse_parts.cuda(), out_dtype=torch.float32)
+    assert ra.device_status() == 0
+    O, L = oracle.lse_merge(torch.nan_to_num(o_parts, nan=0.0), lse_parts)
+    assert torch.isfinite(o).all()
+    assert_close_f32(o.cpu().numpy(), O, tol=1e-5)
+    assert_lse(lse.cpu().numpy(), L, tol=1e-5)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_ring_steps_as_separate_calls_then_merged(ra, causal):
     """The pages' decomposition done literally: each ring position r computes one
