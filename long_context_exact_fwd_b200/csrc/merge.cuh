@@ -23,7 +23,7 @@ namespace merge {
 
 constexpr int WARPS = 8;
 constexpr int CHUNK = 4;          // partials loaded together
-constexpr int BLOCKS_PER_SM = 4;  // resident blocks per SM at the kernel's 64 registers (no spill)
+constexpr int BLOCKS_PER_SM = 8;  // grid cap per SM (4 blocks are resident at 64 registers; the rest queue)
 
 __device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
 __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
