@@ -431,7 +431,7 @@ int ring_attn_merge_ex(const float* o_parts, const float* lse_parts, int P, void
   int st = RA_OK;
   DevInfo* di = dev_info(&st);
   if (!di) return st;
-  // persistent grid: a full SM's worth of blocks per SM, striding over the rows
+  // grid capped at BLOCKS_PER_SM blocks per SM; the kernel strides over the rows
   long long blocks = (rows + ra::merge::WARPS - 1) / ra::merge::WARPS;
   const long long cap = static_cast<long long>(di->sm_count) * ra::merge::BLOCKS_PER_SM;
   if (blocks > cap) blocks = cap;
