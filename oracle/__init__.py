@@ -17,7 +17,10 @@ Parity pins (all in tests/test_oracle*.py, CPU only): brute-force scalar loops o
 inputs, closed forms (identical keys, one-hot scores, causal row 0, constant V, Q=0),
 central finite differences and an independent torch float64 autograd check for the
 backward, merge identities, and order/partition independence of the blockwise ring
-algorithm against the plain definition.  No function here is "parity unpinned".
+algorithm against the plain definition; the key-subset attention against a brute-force
+loop and, over a key partition, merged to the full result; the block-pair gradient with
+full-row statistics summed over block pairs to the full gradient.  No function here is
+"parity unpinned".
 """
 from .attention import (  # noqa: F401
     attn_fwd,
