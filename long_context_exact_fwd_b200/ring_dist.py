@@ -19,6 +19,14 @@ The skipped blocks still travel on, so every rank forwards D - 1 blocks.
 Backward: rank r keeps dQ for its queries; the dK/dV accumulators (fp32) of a key/value block
 travel with that block, collect every rank's contribution, and are back at the block's owner
 after D hops.  The per-block backward uses the global O and lse, so each contribution is exact.
+
+Zig-zag assignment (ring_fwd_zigzag / ring_bwd_zigzag; the striped/zig-zag variant that the
+"Ring Attention" pages name as a follow-up): with contiguous blocks and a causal mask, rank r has
+r + 1 blocks of work and rank D - 1 has D, so the ring waits on the last rank.  Cutting the
+sequence into 2D chunks and giving rank r chunks r and 2D - 1 - r (an early and a late one) gives
+every rank the same work at every ring step: two of the four half-block pairs are visible at every
+step but the first, where three are (two of them on the diagonal).  The ring itself is unchanged;
+only which positions a rank holds, and so which half-block pairs it computes, differ.
 """
 from typing import Callable, Optional, Tuple
 
@@ -167,3 +175,161 @@ def ring_bwd_emulated(q_blocks, k_blocks, v_blocks, o_blocks, lse_blocks, do_blo
             dv[j] += c.float()
     dt = q_blocks[0].dtype
     return [x.to(dt) for x in dq], [x.to(dt) for x in dk], [x.to(dt) for x in dv]
+
+
+def zigzag_chunks(rank: int, world: int) -> Tuple[int, int]:
+    """The two chunks (of 2 * world equal chunks of the sequence) that rank `rank` holds under the
+    zig-zag assignment, in local order: chunk rank, then chunk 2 * world - 1 - rank."""
+    return rank, 2 * world - 1 - rank
+
+
+def zigzag_shard(x: torch.Tensor, rank: int, world: int, dim: int = 2) -> torch.Tensor:
+    """Rank `rank`'s zig-zag shard of a full-sequence tensor (sequence along `dim`): its two
+    chunks concatenated, early chunk first."""
+    S = x.shape[dim]
+    if S % (2 * world):
+        raise ValueError(f"sequence length {S} is not a multiple of 2 * world = {2 * world}")
+    ch = x.chunk(2 * world, dim=dim)
+    a, b = zigzag_chunks(rank, world)
+    return torch.cat((ch[a], ch[b]), dim=dim).contiguous()
+
+
+def zigzag_unshard(shards, dim: int = 2) -> torch.Tensor:
+    """The full-sequence tensor from every rank's zig-zag shard (the inverse of zigzag_shard)."""
+    world = len(shards)
+    chunks = [None] * (2 * world)
+    for r, x in enumerate(shards):
+        a, b = zigzag_chunks(r, world)
+        chunks[a], chunks[b] = x.chunk(2, dim=dim)
+    return torch.cat(chunks, dim=dim)
+
+
+def zigzag_steps(rank: int, world: int, causal: bool):
+    """The work of rank `rank` under the zig-zag assignment, in ring order: (step t, key/value rank
+    j, pairs) for t = 0..world-1 with j = (rank - t) mod world, where pairs lists the half-block
+    pairs (query half a, key/value half b, masked) to compute.  Half a of a rank is its chunk
+    zigzag_chunks(rank)[a].  Causal: a chunk pair is visible when the key chunk does not come
+    after the query chunk, and masked per element when it is the same chunk."""
+    out = []
+    for t in range(world):
+        j = (rank - t) % world
+        qc, kc = zigzag_chunks(rank, world), zigzag_chunks(j, world)
+        pairs = [(a, b, causal and qc[a] == kc[b]) for a in (0, 1) for b in (0, 1)
+                 if not causal or kc[b] <= qc[a]]
+        out.append((t, j, pairs))
+    return out
+
+
+def _halves(x: torch.Tensor):
+    """The two chunks of a zig-zag shard (sequence along dim 2), each contiguous."""
+    if x.shape[2] % 2:
+        raise ValueError(f"a zig-zag shard holds two equal chunks; length {x.shape[2]} is odd")
+    return [h.contiguous() for h in x.chunk(2, dim=2)]
+
+
+def _kv_halves(k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
+    """[half][k or v][B, H, c/2, Dh]: the travelling key/value buffer of a zig-zag shard."""
+    return torch.stack([torch.stack(p) for p in zip(_halves(k), _halves(v))]).contiguous()
+
+
+def _merge_halves(parts, merge):
+    outs = [merge(torch.stack([o for o, _ in p]).contiguous(), torch.stack([l for _, l in p]).contiguous())
+            for p in parts]
+    return torch.cat([o for o, _ in outs], dim=2), torch.cat([l for _, l in outs], dim=2)
+
+
+def ring_fwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, group=None,
+                    block_fwd: Optional[BlockFwd] = None, merge: Optional[Merge] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Forward of this rank's zig-zag shard.  q, k, v: [B, H, c, Dh], zigzag_shard of the full
+    sequence for this rank (c = S / world, even).  Returns (o, lse) in the same shard layout."""
+    ring = _Ring(group)
+    block_fwd = block_fwd or _cuda_block_fwd
+    merge = merge or _cuda_merge
+    qh = _halves(q)
+    kv = _kv_halves(k, v)
+    nxt = torch.empty_like(kv)
+    parts = ([], [])
+    for t, _, pairs in zigzag_steps(ring.rank, ring.world, causal):
+        more = t + 1 < ring.world
+        if more:   # the next shard is in flight while this one is computed
+            ring.start([kv], [nxt])
+        for a, b, masked in pairs:
+            o_t, l_t = block_fwd(qh[a], kv[b, 0], kv[b, 1], masked)
+            parts[a].append((o_t.float(), l_t.float()))
+        if more:
+            ring.wait()
+            kv, nxt = nxt, kv
+    return _merge_halves(parts, merge)
+
+
+def ring_bwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                    do: torch.Tensor, causal: bool = True, group=None, block_bwd: Optional[BlockBwd] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Backward of this rank's zig-zag shard, given ring_fwd_zigzag's o and lse (all tensors in
+    the shard layout).  Returns (dq, dk, dv) in the shard layout, in the dtype of q."""
+    ring = _Ring(group)
+    block_bwd = block_bwd or _cuda_block_bwd
+    qh, oh, lh, dh = _halves(q), _halves(o), _halves(lse), _halves(do)
+    kv = _kv_halves(k, v)
+    g = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)   # dK, dV of the halves held
+    kv_n, g_n = torch.empty_like(kv), torch.empty_like(g)
+    dq = [torch.zeros(h.shape, dtype=torch.float32, device=h.device) for h in qh]
+    for t, _, pairs in zigzag_steps(ring.rank, ring.world, causal):
+        for a, b, masked in pairs:
+            dq_t, dk_t, dv_t = block_bwd(qh[a], kv[b, 0], kv[b, 1], oh[a], lh[a], dh[a], masked)
+            dq[a] += dq_t.float()
+            g[b, 0] += dk_t.float()
+            g[b, 1] += dv_t.float()
+        if ring.world > 1:   # D hops in all: the accumulators end at their shard's owner
+            ring.start([kv, g], [kv_n, g_n])
+            ring.wait()
+            kv, kv_n = kv_n, kv
+            g, g_n = g_n, g
+    dt = q.dtype
+    return (torch.cat(dq, dim=2).to(dt), torch.cat((g[0, 0], g[1, 0]), dim=2).to(dt),
+            torch.cat((g[0, 1], g[1, 1]), dim=2).to(dt))
+
+
+def ring_fwd_zigzag_emulated(q_shards, k_shards, v_shards, causal: bool = True,
+                             block_fwd: Optional[BlockFwd] = None, merge: Optional[Merge] = None):
+    """All ranks of ring_fwd_zigzag in one process, without communication: rank r's (o, lse)
+    from the same zigzag_steps schedule, the shards taken from the lists."""
+    block_fwd = block_fwd or _cuda_block_fwd
+    merge = merge or _cuda_merge
+    world = len(q_shards)
+    kvs = [_kv_halves(k, v) for k, v in zip(k_shards, v_shards)]
+    outs = []
+    for r in range(world):
+        qh = _halves(q_shards[r])
+        parts = ([], [])
+        for _, j, pairs in zigzag_steps(r, world, causal):
+            for a, b, masked in pairs:
+                o_t, l_t = block_fwd(qh[a], kvs[j][b, 0], kvs[j][b, 1], masked)
+                parts[a].append((o_t.float(), l_t.float()))
+        outs.append(_merge_halves(parts, merge))
+    return outs
+
+
+def ring_bwd_zigzag_emulated(q_shards, k_shards, v_shards, o_shards, lse_shards, do_shards, causal: bool = True,
+                             block_bwd: Optional[BlockBwd] = None):
+    """All ranks of ring_bwd_zigzag in one process: dQ of each half summed over its pairs, dK/dV
+    of each key/value half summed over every rank that visits it."""
+    block_bwd = block_bwd or _cuda_block_bwd
+    world = len(q_shards)
+    kvs = [_kv_halves(k, v) for k, v in zip(k_shards, v_shards)]
+    gs = [torch.zeros(kv.shape, dtype=torch.float32, device=kv.device) for kv in kvs]
+    dqs = []
+    for r in range(world):
+        qh, oh, lh, dh = _halves(q_shards[r]), _halves(o_shards[r]), _halves(lse_shards[r]), _halves(do_shards[r])
+        dq = [torch.zeros(h.shape, dtype=torch.float32, device=h.device) for h in qh]
+        for _, j, pairs in zigzag_steps(r, world, causal):
+            for a, b, masked in pairs:
+                dq_t, dk_t, dv_t = block_bwd(qh[a], kvs[j][b, 0], kvs[j][b, 1], oh[a], lh[a], dh[a], masked)
+                dq[a] += dq_t.float()
+                gs[j][b, 0] += dk_t.float()
+                gs[j][b, 1] += dv_t.float()
+        dqs.append(torch.cat(dq, dim=2))
+    dt = q_shards[0].dtype
+    return ([x.to(dt) for x in dqs], [torch.cat((g[0, 0], g[1, 0]), dim=2).to(dt) for g in gs],
+            [torch.cat((g[0, 1], g[1, 1]), dim=2).to(dt) for g in gs])

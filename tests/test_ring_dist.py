@@ -78,6 +78,38 @@ def _rank_main(rank, world, port, causal, out):
     dist.destroy_process_group()
 
 
+def _zigzag_rank_main(rank, world, port, causal, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import oracle
+    from long_context_exact_fwd_b200 import ring_dist as rd
+
+    def block_fwd(q, k, v, masked):
+        return _per_head(lambda a, b, c: oracle.attn_fwd(a, b, c, masked), q, k, v)
+
+    def merge(o_parts, lse_parts):
+        o, l = oracle.lse_merge(o_parts.numpy(), lse_parts.numpy())
+        return torch.from_numpy(o), torch.from_numpy(l)
+
+    def block_bwd(q, k, v, o, lse, do, masked):
+        return _per_head(lambda a, b, c, d, e, f: oracle.attn_bwd_given_stats(a, b, c, d, e, f, masked),
+                         q, k, v, o, lse, do)
+
+    B, H, c, Dh = 1, 2, 6, 4
+    q, k, v, do = _full_inputs(B, H, world * c, Dh, seed=13)
+    sh = lambda x: rd.zigzag_shard(x, rank, world)
+    o, lse = rd.ring_fwd_zigzag(sh(q), sh(k), sh(v), causal, block_fwd=block_fwd, merge=merge)
+    dq, dk, dv = rd.ring_bwd_zigzag(sh(q), sh(k), sh(v), o, lse, sh(do), causal, block_bwd=block_bwd)
+    O, L = _per_head(lambda a, b, cc: oracle.attn_fwd(a, b, cc, causal), q, k, v)
+    dQ, dK, dV = _per_head(lambda a, b, cc, d: oracle.attn_bwd(a, b, cc, d, causal), q, k, v, do)
+    err = lambda x, y: float((x.double() - sh(y)).abs().max())
+    out[rank] = (err(o, O), err(lse, L), err(dq, dQ), err(dk, dK), err(dv, dV))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 @pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("causal", [False, True])
 def test_ring_over_gloo_ranks_matches_the_full_oracle(world, causal):
@@ -102,3 +134,56 @@ def test_ring_steps_follow_the_pages_ring_order():
                 assert [j for _, j, _ in steps] == oracle.ring_order(world, rank, causal)
                 assert [m for _, j, m in steps] == [causal and j == rank for _, j, _ in steps]
                 assert steps[0][:2] == (0, rank)   # own block first
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (4, False), (4, True)])
+def test_zigzag_ring_over_gloo_ranks_matches_the_full_oracle(world, causal):
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_zigzag_rank_main, args=(world, _free_port(), causal, out), nprocs=world, join=True)
+        res = dict(out)
+    assert sorted(res) == list(range(world))
+    for rank, errs in res.items():
+        assert max(errs) < 1e-5, (rank, errs)
+
+
+def test_zigzag_shards_hold_chunks_r_and_2d_minus_1_minus_r():
+    sys.path.insert(0, ROOT)
+    from long_context_exact_fwd_b200 import ring_dist as rd
+    for world in (1, 2, 3, 4, 8):
+        S = 2 * world * 3
+        pos = torch.arange(S).view(1, 1, S, 1).expand(2, 3, S, 5).contiguous()
+        shards = [rd.zigzag_shard(pos, r, world) for r in range(world)]
+        for r, x in enumerate(shards):
+            want = list(range(3 * r, 3 * r + 3)) + list(range(3 * (2 * world - 1 - r), 3 * (2 * world - r)))
+            assert x[1, 2, :, 4].tolist() == want
+            assert x.is_contiguous()
+        assert torch.equal(rd.zigzag_unshard(shards), pos)
+        lse_like = pos[..., 0].contiguous()   # [B, H, S]: the sequence is dim 2 there too
+        assert torch.equal(rd.zigzag_unshard([rd.zigzag_shard(lse_like, r, world) for r in range(world)]), lse_like)
+    with pytest.raises(ValueError):
+        rd.zigzag_shard(torch.zeros(1, 1, 10, 4), 0, 4)
+
+
+def test_zigzag_schedule_covers_every_visible_chunk_pair_once_and_balances_the_steps():
+    sys.path.insert(0, ROOT)
+    from long_context_exact_fwd_b200 import ring_dist as rd
+    for world in range(1, 9):
+        n = 2 * world
+        for causal in (False, True):
+            seen = []
+            for r in range(world):
+                steps = rd.zigzag_steps(r, world, causal)
+                assert [(t, j) for t, j, _ in steps] == [(t, (r - t) % world) for t in range(world)]
+                for t, j, pairs in steps:
+                    qc, kc = rd.zigzag_chunks(r, world), rd.zigzag_chunks(j, world)
+                    seen += [(qc[a], kc[b], m) for a, b, m in pairs]
+                    # work per step in units of one unmasked half-block pair; a masked diagonal
+                    # pair holds half of one
+                    work = sum(0.5 if m else 1.0 for _, _, m in pairs)
+                    assert work == (2.0 if causal else 4.0), (world, r, t, pairs)
+            want = [(a, b, causal and a == b) for a in range(n) for b in range(n) if not causal or b <= a]
+            assert sorted(seen) == sorted(want)
+    # the contiguous assignment, for contrast: rank r has r + 1 blocks of causal work
+    work = [sum(0.5 if m else 1.0 for _, _, m in rd.ring_steps(r, 4, True)) for r in range(4)]
+    assert work == [0.5, 1.5, 2.5, 3.5]

@@ -9,7 +9,8 @@ oracle over the whole sequence.
 Forward bar: the bf16 parity bar (max-abs 2e-2, mean-abs 2e-3, LSE 1e-3).  Backward: each of a
 row's up to D per-step contributions comes back from the library rounded to bf16 and is summed
 in float32, so the bound is (D + 1) half-ulps of bf16 at the largest reference value, with the
-usual mean-abs 2e-3.
+usual mean-abs 2e-3.  The zig-zag ring (ring_fwd_zigzag_emulated / ring_bwd_zigzag_emulated)
+works on half blocks, so a row sums up to 2D contributions: (2D + 1) half-ulps.
 """
 import numpy as np
 import pytest
@@ -52,6 +53,32 @@ def test_emulated_ring_forward_and_backward(rd, causal, D, c):
     for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
         g = torch.cat(got, dim=2).float().cpu().numpy()
         bound = (D + 1) * 2.0 ** -9 * np.abs(want).max()
+        err = np.abs(g - want)
+        assert err.max() <= max(bound, 2e-2), (name, err.max(), bound)
+        assert err.mean() <= 2e-3, (name, err.mean())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D,c", [(2, 384), (4, 256)])
+def test_emulated_zigzag_ring_forward_and_backward(rd, causal, D, c):
+    # zig-zag shards: rank r holds chunks r and 2D - 1 - r of 2D; every half-block pair goes
+    # through the library, so a row's dQ (and a key's dK, dV) sums up to 2D bf16-rounded parts
+    inp = random_qkv(1, 2, D * c, 128, seed=71 + D, with_do=True)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    sh = lambda x: [rd.zigzag_shard(x, r, D) for r in range(D)]
+    outs = rd.ring_fwd_zigzag_emulated(sh(q), sh(k), sh(v), causal)
+    o = rd.zigzag_unshard([x for x, _ in outs])
+    lse = rd.zigzag_unshard([l for _, l in outs])
+    O, L = oracle.attn_fwd_heads(inp["q"], inp["k"], inp["v"], causal)
+    assert_close_bf16(o.float().cpu().numpy(), O, "zig-zag ring o")
+    assert_lse(lse.cpu().numpy(), L)
+
+    dq, dk, dv = rd.ring_bwd_zigzag_emulated(sh(q), sh(k), sh(v), [x for x, _ in outs], [l for _, l in outs],
+                                             sh(do), causal)
+    ref = oracle.attn_bwd_heads(inp["q"], inp["k"], inp["v"], inp["do"], causal)
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        g = rd.zigzag_unshard(got).float().cpu().numpy()
+        bound = (2 * D + 1) * 2.0 ** -9 * np.abs(want).max()
         err = np.abs(g - want)
         assert err.max() <= max(bound, 2e-2), (name, err.max(), bound)
         assert err.mean() <= 2e-3, (name, err.mean())
