@@ -10,6 +10,12 @@ already resident in HBM.  The metric is causal-adjusted TFLOP/s (forward 4*B*H*S
 backward 2.5x forward).  Multi-GPU (torchrun): every rank runs its own seeded replica of
 the workload (weak scaling, no collective on the data path); time is the max over ranks.
 
+End to end ("e2e"): the same steps through the public API with pinned host inputs copied in and
+the step's results (dQ, dK, dV; or O, LSE) copied out every step.  "value" overlaps step i + 1's
+input copies and step i - 1's result copies with step i's compute (two copy streams, two device
+buffer sets), the way a caller streams batches; "serial_value" runs copy in, compute, copy out
+on one stream.  The pipelined results are checked equal to the serial ones.
+
 --impl reference times the float64 CPU oracle on bounded samples of the same workload
 (rank 0 only) and prints the same line shape with "impl": "reference".
 """
