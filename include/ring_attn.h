@@ -127,6 +127,21 @@ RA_API int ring_attn_fwd_split(const void* q, const void* k, const void* v, void
                                ra_stream stream);
 
 /*
+ * ring_attn_fwd_partial -- ring_attn_fwd with a float32 output, for results that are merged
+ * afterwards (page "精读笔记 ...", §3.1: the output over one set of key/value blocks, kept
+ * with its log-sum-exp so that it can be combined with others; the multi-GPU ring merges one
+ * such partial per ring step).
+ *   q, k, v, B, H, S, Dh, D, causal  as ring_attn_fwd (bf16, Dh 64 or 128).
+ *   o_part    [B][H][S][Dh] float32, written: the normalised output O (not rounded to bf16).
+ *   lse_part  [B][H][S] float32, written: natural-log LSE of each row.
+ * Together they are one part of ring_attn_merge's input.  One launch on `stream`.
+ * Errors: RA_ERR_ARG (null pointer), RA_ERR_SHAPE, RA_ERR_ALIGN (q, k, v or o_part not 16-byte
+ * aligned), RA_ERR_CUDA.
+ */
+RA_API int ring_attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B,
+                                 int H, int S, int Dh, int D, int causal, ra_stream stream);
+
+/*
  * ring_attn_bwd_workspace_size -- bytes of device workspace ring_attn_bwd needs: a float32
  * dQ accumulator [B][H][S][Dh] and two float32 row statistics (Delta = rowsum(dO * O) and
  * lse * log2(e)) of [B][H][S_pad] with S_pad = S rounded up to 128, each region 256-byte

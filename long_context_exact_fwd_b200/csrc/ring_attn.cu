@@ -139,8 +139,9 @@ int launch_status() {
   return e == cudaSuccess ? RA_OK : cuda_fail(static_cast<int>(e), "kernel launch");
 }
 
-// n_parts > 1: each query pair's visit order is cut into n_parts pieces, written as fp32
-// partials to o_part / lse_part ([n_parts][B*H][S][HD], [n_parts][B*H][S]) for the merge.
+// o_part given: each query pair's visit order is cut into n_parts pieces (n_parts >= 1),
+// written as fp32 partials to o_part / lse_part ([n_parts][B*H][S][HD], [n_parts][B*H][S])
+// for the merge; o and lse are then not written.
 template <int HD>
 int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D, int causal,
              float scale, cudaStream_t stream, int n_parts = 1, float* o_part = nullptr, float* lse_part = nullptr) {
@@ -173,7 +174,7 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.o_part = o_part;
   p.lse_part = lse_part;
   constexpr int smem = Layout<HD>::ALLOC;
-  const bool split = n_parts > 1;
+  const bool split = o_part != nullptr;
   const int slot = (HD == 128 ? 0 : 1) + (split ? 2 : 0);
   auto kern = split ? fwd_kernel<HD, true> : fwd_kernel<HD, false>;
   if (!di->fwd_attr[slot]) {
@@ -417,6 +418,20 @@ int ring_attn_fwd_split(const void* q, const void* k, const void* v, void* o, fl
                  : fwd_bf16<64>(q, k, v, o, lse, B, H, S, D, causal, sc, s, n_parts, o_part, lse_part);
   if (st != RA_OK) return st;
   return ring_attn_merge(o_part, lse_part, n_parts, o, lse, B, H, S, Dh, stream);
+}
+
+int ring_attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int H,
+                          int S, int Dh, int D, int causal, ra_stream stream) {
+  if (!q || !k || !v || !o_part || !lse_part) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  if (Dh != 128 && Dh != 64) return RA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part)) return RA_ERR_ALIGN;
+  const float sc = 1.f / std::sqrt(static_cast<float>(Dh));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // one piece: the split kernel's fp32 epilogue over the whole visit order
+  return Dh == 128 ? fwd_bf16<128>(q, k, v, nullptr, nullptr, B, H, S, D, causal, sc, s, 1, o_part, lse_part)
+                   : fwd_bf16<64>(q, k, v, nullptr, nullptr, B, H, S, D, causal, sc, s, 1, o_part, lse_part);
 }
 
 int ring_attn_merge_ex(const float* o_parts, const float* lse_parts, int P, void* o, float* lse, int B, int H, int S,

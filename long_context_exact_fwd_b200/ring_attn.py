@@ -39,6 +39,7 @@ _fwd_ex = _sig("ring_attn_fwd_ex", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, 
 _bwd_ws = _sig("ring_attn_bwd_workspace_size", _sz, _i, _i, _i, _i)
 _split_ws = _sig("ring_attn_fwd_split_workspace_size", _sz, _i, _i, _i, _i, _i)
 _fwd_split = _sig("ring_attn_fwd_split", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
+_fwd_partial = _sig("ring_attn_fwd_partial", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _bwd = _sig("ring_attn_bwd", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
 _merge_ex = _sig("ring_attn_merge_ex", _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp)
 _ring_order = _sig("ring_attn_ring_order", _i, _i, _i, _i, _ip, _i)
@@ -172,6 +173,26 @@ def fwd_split(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, D: int, causal:
                       1 if causal else 0, n_parts, workspace.data_ptr(),
                       workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "ring_attn_fwd_split")
+    return out, lse
+
+
+def fwd_partial(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, D: int, causal: bool = True,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Forward with a float32 output (ring_attn_fwd_partial): (o [B, H, S, Dh] f32, lse
+    [B, H, S] f32), one part for merge().  q, k, v: [B, H, S, Dh] bf16."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, S, Dh]")
+    B, H, S, Dh = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, q.shape)
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device) if out is None else out
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(out, "out", torch.float32, q.shape)
+    _need(lse, "lse", torch.float32, (B, H, S))
+    code = _fwd_partial(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, S, Dh, D,
+                        1 if causal else 0, _stream(stream))
+    _check(code, "ring_attn_fwd_partial")
     return out, lse
 
 

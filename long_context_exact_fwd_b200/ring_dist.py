@@ -8,8 +8,8 @@ it currently holds.  At ring step t rank r holds block (r - t) mod D (its own bl
 §3.5 walk-through); the transfer of the next block is posted before the compute of the current
 one, so the two overlap (§3.3).  Partial results combine through their log-sum-exp (§3.1).
 
-The per-block work runs in the CUDA library (ring_attn_fwd / ring_attn_bwd on one block pair,
-ring_attn_merge for the partials); this module is host orchestration only: torch.distributed
+The per-block work runs in the CUDA library (ring_attn_fwd_partial / ring_attn_bwd on one block
+pair, ring_attn_merge for the partials: each step's forward output stays float32 until the merge); this module is host orchestration only: torch.distributed
 point-to-point sends and receives between neighbours (NCCL over NVLink on GPUs), no collective.
 
 Causal masking is on global positions: block j is entirely visible to block r when j < r, masked
@@ -40,7 +40,7 @@ Merge = Callable[[torch.Tensor, torch.Tensor], Tuple[torch.Tensor, torch.Tensor]
 
 def _cuda_block_fwd(q, k, v, causal):
     from . import ring_attn as ra
-    return ra.fwd(q, k, v, 1, causal)
+    return ra.fwd_partial(q, k, v, 1, causal)   # float32 partial, rounded to bf16 only by the merge
 
 
 def _cuda_block_bwd(q, k, v, o, lse, do, causal):

@@ -96,6 +96,22 @@ def test_split_forward_workspace_and_argument_errors(ra):
     assert f(*args(q=24)) == ra.RA_ERR_ALIGN
 
 
+def test_partial_forward_argument_errors(ra):
+    f = ra.raw.ring_attn_fwd_partial
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    args = lambda **kw: [P(kw.get("q", 256)), P(256), P(256), P(kw.get("o", 256)), P(kw.get("lse", 256)), 1, 2,
+                         kw.get("S", 1024), kw.get("Dh", 128), kw.get("D", 4), 1, P(0)]
+    # all rejected before anything is enqueued (no device needed)
+    assert f(*args(q=0)) == ra.RA_ERR_ARG
+    assert f(*args(o=0)) == ra.RA_ERR_ARG
+    assert f(*args(lse=0)) == ra.RA_ERR_ARG
+    assert f(*args(S=1000, D=3)) == ra.RA_ERR_SHAPE      # S % D != 0
+    assert f(*args(Dh=96)) == ra.RA_ERR_SHAPE
+    assert f(*args(q=24)) == ra.RA_ERR_ALIGN
+    assert f(*args(o=264)) == ra.RA_ERR_ALIGN
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_library_ring_order_matches_oracle(ra, causal):
     for D in (1, 2, 3, 4, 7, 8, 16):

@@ -2,8 +2,8 @@
 
 ring_dist.ring_fwd_emulated / ring_bwd_emulated run every rank of a D-rank ring in one process
 with the same ring_steps schedule as the distributed ring_fwd / ring_bwd (no communication: the
-blocks come from lists), so each block pair goes through ring_attn_fwd / ring_attn_bwd with the
-mask the ring gives it, and the partials through ring_attn_merge.  Compared with the float64
+blocks come from lists), so each block pair goes through ring_attn_fwd_partial (float32 partial) /
+ring_attn_bwd with the mask the ring gives it, and the partials through ring_attn_merge.  Compared with the float64
 oracle over the whole sequence.
 
 Forward bar: the bf16 parity bar (max-abs 2e-2, mean-abs 2e-3, LSE 1e-3).  Backward: each of a

@@ -141,3 +141,22 @@ def test_auto_parts_choice(ra):
     O, L = oracle.attn_fwd_heads(inp["q"], inp["k"], inp["v"], True)
     assert_close_bf16(o.float().cpu().numpy(), O)
     assert_lse(lse.cpu().numpy(), L)
+
+
+@pytest.mark.parametrize("B,H,S,Dh,D", SPLIT_SHAPES)
+@pytest.mark.parametrize("causal", [False, True])
+def test_partial_forward_is_the_plain_forward_in_float32(ra, B, H, S, Dh, D, causal):
+    # ring_attn_fwd_partial: the whole ring as one float32 part; merged alone it must give the
+    # bf16 forward bit for bit (weight exp(0) = 1, one rounding to bf16 in both)
+    inp = random_qkv(B, H, S, Dh, seed=90 + S % 97 + D)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o32, l32 = ra.fwd_partial(q, k, v, D, causal)
+    o16, l16 = ra.fwd(q, k, v, D, causal)
+    assert o32.dtype == torch.float32 and ra.device_status() == 0
+    O, L = oracle.attn_fwd_heads(inp["q"], inp["k"], inp["v"], causal)
+    assert_close_bf16(o32.cpu().numpy(), O, "fp32 partial o")
+    assert_lse(l32.cpu().numpy(), L)
+    om, lm = ra.merge(o32[None].contiguous(), l32[None].contiguous())
+    assert torch.equal(om, o16)
+    assert torch.allclose(lm, l16, atol=1e-6, rtol=0)
+    assert torch.equal(o32.to(torch.bfloat16), o16)
