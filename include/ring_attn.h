@@ -169,6 +169,23 @@ RA_API int ring_attn_bwd(const void* q, const void* k, const void* v, const void
                   size_t workspace_bytes, ra_stream stream);
 
 /*
+ * ring_attn_bwd_accumulate -- ring_attn_bwd whose gradients are added, in float32, to the
+ * caller's accumulators instead of written in bf16: dq32 += dQ, dk32 += dK, dv32 += dV.  For
+ * gradients summed over several calls (the multi-GPU ring: dQ of a rank's queries over the
+ * ring steps, dK and dV of a travelling key/value block over the ranks; page "精读笔记 ...",
+ * §4.2: training runs through the same blockwise ring), rounded once by the caller at the end.
+ *   q, k, v, o, lse, dO, B, H, S, Dh, D, causal, workspace  as ring_attn_bwd.
+ *   dq32, dk32, dv32  [B][H][S][Dh] float32, 16-byte aligned, read and written; the caller
+ *                     clears them before the first call.
+ * Launches as ring_attn_bwd, with the last one adding the scaled dQ instead of converting it.
+ * Errors as ring_attn_bwd.
+ */
+RA_API int ring_attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                    const void* dO, float* dq32, float* dk32, float* dv32, int B, int H, int S,
+                                    int Dh, int D, int causal, void* workspace, size_t workspace_bytes,
+                                    ra_stream stream);
+
+/*
  * ring_attn_bwd_noalloc -- ring_attn_bwd for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point; it exists for callers that may not call
  * cudaMalloc (or any allocator) on their path -- for example code embedded in a host

@@ -111,6 +111,8 @@ struct Params {
   float* dq_acc;         // [BH][S][HD] fp32
   __nv_bfloat16* dk;     // [BH][S][HD]
   __nv_bfloat16* dv;
+  float* dk32;           // non-null: dK, dV are added to these fp32 [BH][S][HD] instead of
+  float* dv32;           // written to dk, dv (rows of a key tile belong to one CTA)
 };
 
 using RingQTiles = ::ra::RingQTiles;
@@ -418,6 +420,21 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
         uint32_t rr[32];
         tmem_ld32(lane_base + col + 32 * c, rr);
         tmem_ld_wait();
+        if (p.dk32 != nullptr) {   // uniform: accumulate in fp32
+          if (row_ok) {
+            float4* acc = reinterpret_cast<float4*>((which ? p.dk32 : p.dv32) + off + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 a = acc[i];
+              a.x = fmaf(__uint_as_float(rr[4 * i]), mul, a.x);
+              a.y = fmaf(__uint_as_float(rr[4 * i + 1]), mul, a.y);
+              a.z = fmaf(__uint_as_float(rr[4 * i + 2]), mul, a.z);
+              a.w = fmaf(__uint_as_float(rr[4 * i + 3]), mul, a.w);
+              acc[i] = a;
+            }
+          }
+          continue;
+        }
         uint32_t w16[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -624,6 +641,20 @@ __global__ void __launch_bounds__(256)
   const float4 b = __ldg(reinterpret_cast<const float4*>(dq_acc) + 2 * i + 1);
   reinterpret_cast<uint4*>(dq)[i] = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
                                                pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+}
+
+// dQ32 += scale * accumulator (fp32), 4 elements per thread.
+__global__ void __launch_bounds__(256)
+    bwd_accum_dq_kernel(const float* __restrict__ dq_acc, float* __restrict__ dq32, long long n4, float scale) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 a = __ldg(reinterpret_cast<const float4*>(dq_acc) + i);
+  float4 d = reinterpret_cast<const float4*>(dq32)[i];
+  d.x = fmaf(a.x, scale, d.x);
+  d.y = fmaf(a.y, scale, d.y);
+  d.z = fmaf(a.z, scale, d.z);
+  d.w = fmaf(a.w, scale, d.w);
+  reinterpret_cast<float4*>(dq32)[i] = d;
 }
 
 }  // namespace bwd

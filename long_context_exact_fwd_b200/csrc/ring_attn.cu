@@ -224,9 +224,11 @@ BwdWorkspace bwd_workspace(long long BH, int S, int Dh) {
   return w;
 }
 
+// dq32 given: dQ, dK, dV are added to the fp32 dq32, dk32, dv32 instead of written to the
+// bf16 dq, dk, dv.
 int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
              void* dk, void* dv, int B, int H, int S, int D, int causal, float scale, void* workspace,
-             cudaStream_t stream) {
+             cudaStream_t stream, float* dq32 = nullptr, float* dk32 = nullptr, float* dv32 = nullptr) {
   namespace rb = ra::bwd;
   int st = RA_OK;
   DevInfo* di = dev_info(&st);
@@ -274,6 +276,8 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   p.dq_acc = dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk32 = dq32 ? dk32 : nullptr;
+  p.dv32 = dq32 ? dv32 : nullptr;
   constexpr int smem = rb::Layout::BYTES;
   if (!di->bwd_attr) {
     const cudaError_t e = cudaFuncSetAttribute(rb::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -284,7 +288,14 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   rb::bwd_kernel<<<grid, rb::NUM_THREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
   if ((st = launch_status()) != RA_OK) return st;
 
-  // 3. dQ = scale * accumulator -> bf16
+  // 3. dQ = scale * accumulator -> bf16 (or added to dq32)
+  if (dq32) {
+    const long long n4 = BH * S * rb::HD / 4;
+    const long long ablocks = (n4 + 255) / 256;
+    if (ablocks > INT_MAX) return RA_ERR_SHAPE;
+    rb::bwd_accum_dq_kernel<<<static_cast<int>(ablocks), 256, 0, stream>>>(dq_acc, dq32, n4, scale);
+    return launch_status();
+  }
   const long long n8 = BH * S * rb::HD / 8;
   const long long cblocks = (n8 + 255) / 256;
   if (cblocks > INT_MAX) return RA_ERR_SHAPE;
@@ -527,6 +538,24 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* o, co
   const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
   return bwd_bf16(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, workspace,
                   static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, float* dq32, float* dk32, float* dv32, int B, int H, int S, int Dh, int D,
+                             int causal, void* workspace, size_t workspace_bytes, ra_stream stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq32 || !dk32 || !dv32) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  if (Dh != ra::bwd::HD) return RA_ERR_SHAPE;
+  for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(dq32), static_cast<const void*>(dk32),
+                          static_cast<const void*>(dv32)})
+    if (!aligned16(ptr)) return RA_ERR_ALIGN;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < ring_attn_bwd_workspace_size(B, H, S, Dh))
+    return RA_ERR_WORKSPACE;
+  const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
+  return bwd_bf16(q, k, v, o, lse, dO, nullptr, nullptr, nullptr, B, H, S, D, causal, sc, workspace,
+                  static_cast<cudaStream_t>(stream), dq32, dk32, dv32);
 }
 
 int ring_attn_bwd_visit_tiles(int S, int D, int causal, int k0, int tile_rows, int* tiles, int max_tiles) {

@@ -50,6 +50,8 @@ _version = _sig("ring_attn_version", _i)
 _last_cuda = _sig("ring_attn_last_cuda_error", _i, ctypes.POINTER(ctypes.c_char_p))
 _bwd_visit_tiles = _sig("ring_attn_bwd_visit_tiles", _i, _i, _i, _i, _i, _i, _ip, _i)
 _launch_count = _sig("ring_attn_launch_count", ctypes.c_ulonglong)
+_bwd_acc = _sig("ring_attn_bwd_accumulate", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                _i, _vp, _sz, _vp)
 _bwd_noalloc = _sig("ring_attn_bwd_noalloc", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _noalloc_max = _sig("ring_attn_bwd_noalloc_max_bytes", _sz)
 _exp2_check = _sig("ring_attn_exp2_check", _i, _vp, _vp, _vp, ctypes.c_longlong, _vp)
@@ -221,6 +223,28 @@ def bwd(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=N
                 workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "ring_attn_bwd")
     return dq, dk, dv
+
+
+def bwd_accumulate(q, k, v, o, lse, do, D: int, causal: bool, dq32: torch.Tensor, dk32: torch.Tensor,
+                   dv32: torch.Tensor, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward whose gradients are added to float32 accumulators (ring_attn_bwd_accumulate):
+    dq32 += dQ, dk32 += dK, dv32 += dV, each [B, H, S, Dh] float32 cleared by the caller
+    before the first call."""
+    B, H, S, Dh = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, name, torch.bfloat16, q.shape)
+    _need(lse, "lse", torch.float32, (B, H, S))
+    for name, t in (("dq32", dq32), ("dk32", dk32), ("dv32", dv32)):
+        _need(t, name, torch.float32, q.shape)
+    need = bwd_workspace_bytes(B, H, S, Dh)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    code = _bwd_acc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                    dq32.data_ptr(), dk32.data_ptr(), dv32.data_ptr(), B, H, S, Dh, D, 1 if causal else 0,
+                    workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "ring_attn_bwd_accumulate")
+    return dq32, dk32, dv32
 
 
 def bwd_noalloc(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=None, stream=None):

@@ -8,8 +8,9 @@ it currently holds.  At ring step t rank r holds block (r - t) mod D (its own bl
 §3.5 walk-through); the transfer of the next block is posted before the compute of the current
 one, so the two overlap (§3.3).  Partial results combine through their log-sum-exp (§3.1).
 
-The per-block work runs in the CUDA library (ring_attn_fwd_partial / ring_attn_bwd on one block
-pair, ring_attn_merge for the partials: each step's forward output stays float32 until the merge); this module is host orchestration only: torch.distributed
+The per-block work runs in the CUDA library (ring_attn_fwd_partial / ring_attn_bwd_accumulate on
+one block pair, ring_attn_merge for the partials: each step's forward output and gradients stay
+float32 until the end); this module is host orchestration only: torch.distributed
 point-to-point sends and receives between neighbours (NCCL over NVLink on GPUs), no collective.
 
 Causal masking is on global positions: block j is entirely visible to block r when j < r, masked
@@ -43,9 +44,23 @@ def _cuda_block_fwd(q, k, v, causal):
     return ra.fwd_partial(q, k, v, 1, causal)   # float32 partial, rounded to bf16 only by the merge
 
 
-def _cuda_block_bwd(q, k, v, o, lse, do, causal):
+def _cuda_block_bwd_acc(q, k, v, o, lse, do, causal, dq32, dk32, dv32):
     from . import ring_attn as ra
-    return ra.bwd(q, k, v, o, lse, do, 1, causal)
+    ra.bwd_accumulate(q, k, v, o, lse, do, 1, causal, dq32, dk32, dv32)   # float32, added in place
+
+
+def _accumulating(block_bwd: Optional[BlockBwd]):
+    """A block backward that adds its gradients to float32 accumulators: the library's
+    (ring_attn_bwd_accumulate) by default, else one adding what `block_bwd` returns."""
+    if block_bwd is None:
+        return _cuda_block_bwd_acc
+
+    def acc(q, k, v, o, lse, do, causal, dq32, dk32, dv32):
+        a, b, c = block_bwd(q, k, v, o, lse, do, causal)
+        dq32 += a.to(dq32.dtype)
+        dk32 += b.to(dk32.dtype)
+        dv32 += c.to(dv32.dtype)
+    return acc
 
 
 def _cuda_merge(o_parts, lse_parts):
@@ -122,7 +137,7 @@ def ring_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     """Backward of this rank's blocks, given the ring forward's o and lse.  Returns
     (dq, dk, dv) for this rank's block, in the dtype of q."""
     ring = _Ring(group)
-    block_bwd = block_bwd or _cuda_block_bwd
+    block_acc = _accumulating(block_bwd)
     kv = torch.stack((k, v)).contiguous()
     g = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)   # dK, dV of the block held
     kv_n, g_n = torch.empty_like(kv), torch.empty_like(g)
@@ -130,10 +145,7 @@ def ring_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     work = {t: masked for t, _, masked in ring_steps(ring.rank, ring.world, causal)}
     for t in range(ring.world):
         if t in work:
-            dq_t, dk_t, dv_t = block_bwd(q, kv[0], kv[1], o, lse, do, work[t])
-            dq += dq_t.float()
-            g[0] += dk_t.float()
-            g[1] += dv_t.float()
+            block_acc(q, kv[0], kv[1], o, lse, do, work[t], dq, g[0], g[1])
         if ring.world > 1:   # D hops in all: the accumulators end at their block's owner
             ring.start([kv, g], [kv_n, g_n])
             ring.wait()
@@ -162,17 +174,15 @@ def ring_bwd_emulated(q_blocks, k_blocks, v_blocks, o_blocks, lse_blocks, do_blo
                       block_bwd: Optional[BlockBwd] = None):
     """All ranks of ring_bwd in one process: dQ of block r summed over its steps, dK/dV of block
     j summed over every rank that visits it (what the travelling accumulators collect)."""
-    block_bwd = block_bwd or _cuda_block_bwd
+    block_acc = _accumulating(block_bwd)
     world = len(q_blocks)
     dq = [torch.zeros(b.shape, dtype=torch.float32, device=b.device) for b in q_blocks]
     dk = [torch.zeros(b.shape, dtype=torch.float32, device=b.device) for b in k_blocks]
     dv = [torch.zeros(b.shape, dtype=torch.float32, device=b.device) for b in v_blocks]
     for r in range(world):
         for _, j, masked in ring_steps(r, world, causal):
-            a, b, c = block_bwd(q_blocks[r], k_blocks[j], v_blocks[j], o_blocks[r], lse_blocks[r], do_blocks[r], masked)
-            dq[r] += a.float()
-            dk[j] += b.float()
-            dv[j] += c.float()
+            block_acc(q_blocks[r], k_blocks[j], v_blocks[j], o_blocks[r], lse_blocks[r], do_blocks[r], masked,
+                      dq[r], dk[j], dv[j])
     dt = q_blocks[0].dtype
     return [x.to(dt) for x in dq], [x.to(dt) for x in dk], [x.to(dt) for x in dv]
 
@@ -269,7 +279,7 @@ def ring_bwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.
     """Backward of this rank's zig-zag shard, given ring_fwd_zigzag's o and lse (all tensors in
     the shard layout).  Returns (dq, dk, dv) in the shard layout, in the dtype of q."""
     ring = _Ring(group)
-    block_bwd = block_bwd or _cuda_block_bwd
+    block_acc = _accumulating(block_bwd)
     qh, oh, lh, dh = _halves(q), _halves(o), _halves(lse), _halves(do)
     kv = _kv_halves(k, v)
     g = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)   # dK, dV of the halves held
@@ -277,10 +287,7 @@ def ring_bwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.
     dq = [torch.zeros(h.shape, dtype=torch.float32, device=h.device) for h in qh]
     for t, _, pairs in zigzag_steps(ring.rank, ring.world, causal):
         for a, b, masked in pairs:
-            dq_t, dk_t, dv_t = block_bwd(qh[a], kv[b, 0], kv[b, 1], oh[a], lh[a], dh[a], masked)
-            dq[a] += dq_t.float()
-            g[b, 0] += dk_t.float()
-            g[b, 1] += dv_t.float()
+            block_acc(qh[a], kv[b, 0], kv[b, 1], oh[a], lh[a], dh[a], masked, dq[a], g[b, 0], g[b, 1])
         if ring.world > 1:   # D hops in all: the accumulators end at their shard's owner
             ring.start([kv, g], [kv_n, g_n])
             ring.wait()
@@ -315,7 +322,7 @@ def ring_bwd_zigzag_emulated(q_shards, k_shards, v_shards, o_shards, lse_shards,
                              block_bwd: Optional[BlockBwd] = None):
     """All ranks of ring_bwd_zigzag in one process: dQ of each half summed over its pairs, dK/dV
     of each key/value half summed over every rank that visits it."""
-    block_bwd = block_bwd or _cuda_block_bwd
+    block_acc = _accumulating(block_bwd)
     world = len(q_shards)
     kvs = [_kv_halves(k, v) for k, v in zip(k_shards, v_shards)]
     gs = [torch.zeros(kv.shape, dtype=torch.float32, device=kv.device) for kv in kvs]
@@ -325,10 +332,8 @@ def ring_bwd_zigzag_emulated(q_shards, k_shards, v_shards, o_shards, lse_shards,
         dq = [torch.zeros(h.shape, dtype=torch.float32, device=h.device) for h in qh]
         for _, j, pairs in zigzag_steps(r, world, causal):
             for a, b, masked in pairs:
-                dq_t, dk_t, dv_t = block_bwd(qh[a], kvs[j][b, 0], kvs[j][b, 1], oh[a], lh[a], dh[a], masked)
-                dq[a] += dq_t.float()
-                gs[j][b, 0] += dk_t.float()
-                gs[j][b, 1] += dv_t.float()
+                block_acc(qh[a], kvs[j][b, 0], kvs[j][b, 1], oh[a], lh[a], dh[a], masked, dq[a], gs[j][b, 0],
+                          gs[j][b, 1])
         dqs.append(torch.cat(dq, dim=2))
     dt = q_shards[0].dtype
     return ([x.to(dt) for x in dqs], [torch.cat((g[0, 0], g[1, 0]), dim=2).to(dt) for g in gs],

@@ -112,6 +112,25 @@ def test_partial_forward_argument_errors(ra):
     assert f(*args(o=264)) == ra.RA_ERR_ALIGN
 
 
+def test_accumulating_backward_argument_errors(ra):
+    f = ra.raw.ring_attn_bwd_accumulate
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    args = lambda **kw: [P(kw.get("q", 256))] + [P(256)] * 5 + [P(kw.get("dq32", 256)), P(256), P(256), 1, 2,
+                                                                 kw.get("S", 1024), kw.get("Dh", 128), 4, 1,
+                                                                 P(kw.get("ws", 256)),
+                                                                 ctypes.c_size_t(kw.get("ws_bytes", 1 << 40)), P(0)]
+    # all rejected before anything is enqueued (no device needed)
+    assert f(*args(q=0)) == ra.RA_ERR_ARG
+    assert f(*args(dq32=0)) == ra.RA_ERR_ARG
+    assert f(*args(S=1001)) == ra.RA_ERR_SHAPE
+    assert f(*args(Dh=64)) == ra.RA_ERR_SHAPE          # the backward is Dh = 128 only
+    assert f(*args(dq32=264)) == ra.RA_ERR_ALIGN
+    assert f(*args(ws=0)) == ra.RA_ERR_WORKSPACE
+    assert f(*args(ws=272)) == ra.RA_ERR_WORKSPACE
+    assert f(*args(ws_bytes=1024)) == ra.RA_ERR_WORKSPACE
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_library_ring_order_matches_oracle(ra, causal):
     for D in (1, 2, 3, 4, 7, 8, 16):
