@@ -15,8 +15,10 @@ pages leave open are listed in the module docstrings.
 
 Parity pins (all in tests/test_oracle*.py, CPU only): brute-force scalar loops on tiny
 inputs, closed forms (identical keys, one-hot scores, causal row 0, constant V, Q=0),
-central finite differences and an independent torch float64 autograd check for the
-backward, merge identities, and order/partition independence of the blockwise ring
+invariances (linearity in V with the LSE independent of V, key/value and query
+permutations without a mask, a common shift of all keys moving each LSE by its score
+offset), central finite differences, an independent torch float64 autograd check and
+linearity in dO for the backward, merge identities, and order/partition independence of the blockwise ring
 algorithm against the plain definition; the key-subset attention against a brute-force
 loop and, over a key partition, merged to the full result; the block-pair gradient with
 full-row statistics summed over block pairs to the full gradient.  No function here is

@@ -207,7 +207,60 @@ def test_explicit_scale_overrides_default():
     np.testing.assert_allclose(L1, L2, atol=1e-14)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_output_is_linear_in_v_and_lse_does_not_depend_on_v(causal):
+    # O is a convex combination of V rows with weights fixed by Q and K
+    S, Dh = 11, 5
+    q, k, v1, v2 = (_rand((S, Dh), s) for s in (33, 34, 35, 36))
+    O1, L1 = attn_fwd(q, k, v1, causal)
+    O2, L2 = attn_fwd(q, k, v2, causal)
+    O3, L3 = attn_fwd(q, k, 2.5 * v1 - 0.75 * v2, causal)
+    np.testing.assert_allclose(O3, 2.5 * O1 - 0.75 * O2, atol=1e-13)
+    np.testing.assert_allclose(L3, L1, atol=0)
+    np.testing.assert_allclose(L2, L1, atol=0)
+
+
+def test_permutations_of_keys_and_queries():
+    # without a mask, attention is a function of the set of (key, value) pairs and acts row by
+    # row on the queries
+    S, Dh = 12, 4
+    q, k, v = (_rand((S, Dh), s) for s in (37, 38, 39))
+    O, L = attn_fwd(q, k, v, False)
+    pk = np.random.default_rng(40).permutation(S)
+    Ok, Lk = attn_fwd(q, k[pk], v[pk], False)
+    np.testing.assert_allclose(Ok, O, atol=1e-13)
+    np.testing.assert_allclose(Lk, L, atol=1e-13)
+    pq = np.random.default_rng(41).permutation(S)
+    Oq, Lq = attn_fwd(q[pq], k, v, False)
+    np.testing.assert_allclose(Oq, O[pq], atol=1e-14)
+    np.testing.assert_allclose(Lq, L[pq], atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_shifting_every_key_shifts_each_lse_by_its_score_offset(causal):
+    # k_j + u adds scale * q_i . u to every visible score of row i: O unchanged,
+    # LSE_i + scale * q_i . u
+    S, Dh = 9, 6
+    q, k, v = (_rand((S, Dh), s) for s in (42, 43, 44))
+    u = _rand((Dh,), 45)
+    O, L = attn_fwd(q, k, v, causal)
+    Os, Ls = attn_fwd(q, k + u, v, causal)
+    np.testing.assert_allclose(Os, O, atol=1e-13)
+    np.testing.assert_allclose(Ls, L + (q @ u) / math.sqrt(Dh), atol=1e-13)
+
+
 # ---------------------------------------------------------------- backward
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_is_linear_in_do(causal):
+    S, Dh = 10, 4
+    q, k, v, do1, do2 = (_rand((S, Dh), s) for s in (46, 47, 48, 49, 50))
+    g1 = attn_bwd(q, k, v, do1, causal)
+    g2 = attn_bwd(q, k, v, do2, causal)
+    g3 = attn_bwd(q, k, v, -1.5 * do1 + 0.5 * do2, causal)
+    for a, b, c in zip(g1, g2, g3):
+        np.testing.assert_allclose(c, -1.5 * a + 0.5 * b, atol=1e-12)
+
+
 def _loss(q, k, v, do, causal):
     O, _ = attn_fwd(q, k, v, causal)
     return float((O * do).sum())
