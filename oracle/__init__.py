@@ -21,7 +21,9 @@ offset), central finite differences, an independent torch float64 autograd check
 linearity in dO for the backward, merge identities, and order/partition independence of the blockwise ring
 algorithm against the plain definition; the key-subset attention against a brute-force
 loop and, over a key partition, merged to the full result; the block-pair gradient with
-full-row statistics summed over block pairs to the full gradient.  No function here is
+full-row statistics summed over block pairs to the full gradient; the per-head wrappers
+(forward and backward) against per-slice calls and, for the backward over several batch
+entries and heads, against batched torch float64 autograd.  No function here is
 "parity unpinned".
 """
 from .attention import (  # noqa: F401

@@ -419,3 +419,46 @@ def test_heads_wrapper_accepts_bf16_torch_inputs():
                       t["v"][0, 1].double().numpy(), True)
     np.testing.assert_allclose(O[0, 1], O0, atol=0)
     np.testing.assert_allclose(L[0, 1], L0, atol=0)
+
+
+def _torch_batched_grads(q, k, v, do, causal, scale):
+    """float64 autograd of the plain batched formula over [B, H, S, Dh] (a library check
+    independent of the oracle's per-head code)."""
+    qt, kt, vt = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    s = torch.einsum("bhid,bhjd->bhij", qt, kt) * scale
+    if causal:
+        S = s.shape[-1]
+        s = s.masked_fill(torch.ones(S, S, dtype=torch.bool).triu(1), float("-inf"))
+    o = torch.einsum("bhij,bhjd->bhid", torch.softmax(s, dim=-1), vt)
+    (o * torch.tensor(do, dtype=torch.float64)).sum().backward()
+    return qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_heads_wrapper_matches_batched_autograd(causal):
+    """attn_bwd_heads over [B=2, H=3]: every head equals batched float64 autograd (catches a
+    head-index or batch/head transposition slip), with a non-default scale passed through."""
+    B, H, S, Dh = 2, 3, 11, 5
+    q, k, v, do = (_rand((B, H, S, Dh), s) for s in (61, 62, 63, 64))
+    sc = 0.37
+    dq, dk, dv = oracle.attn_bwd_heads(q, k, v, do, causal, scale=sc)
+    tq, tk, tv = _torch_batched_grads(q, k, v, do, causal, sc)
+    np.testing.assert_allclose(dq, tq, atol=1e-12)
+    np.testing.assert_allclose(dk, tk, atol=1e-12)
+    np.testing.assert_allclose(dv, tv, atol=1e-12)
+
+
+def test_bwd_heads_wrapper_filters_heads_and_accepts_bf16_torch_inputs():
+    """Listed heads equal attn_bwd on that head's float64 slices exactly; unlisted heads are NaN."""
+    from long_context_exact_fwd_b200.workloads import random_qkv
+    t = random_qkv(2, 3, 16, 8, seed=5, with_do=True)
+    heads = [(0, 2), (1, 0)]
+    dq, dk, dv = oracle.attn_bwd_heads(t["q"], t["k"], t["v"], t["do"], True, heads=heads)
+    for b in range(2):
+        for h in range(3):
+            if (b, h) in heads:
+                ref = attn_bwd(*(t[n][b, h].double().numpy() for n in ("q", "k", "v", "do")), True)
+                for got, want in zip((dq, dk, dv), ref):
+                    np.testing.assert_allclose(got[b, h], want, atol=0)
+            else:
+                assert np.isnan(dq[b, h]).all() and np.isnan(dk[b, h]).all() and np.isnan(dv[b, h]).all()
