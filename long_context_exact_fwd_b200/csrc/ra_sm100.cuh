@@ -297,7 +297,9 @@ __device__ __forceinline__ float exp2_fma(float x) {
   const float t = __fadd_rn(x, 12582912.f);
   const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
   const float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  // unsigned arithmetic: the shift moves bits of the 1.5 * 2^23 offset past bit 31, which
+  // is well defined only on unsigned values; the wrap-around leaves exactly n << 23
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // Two lanes of exp2_fma with packed f32x2 arithmetic (same polynomial, same bound).
@@ -310,8 +312,8 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
   float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
   p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
   p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Three-input maximum (one instruction on sm_100).

@@ -56,8 +56,10 @@ struct DevInfo {
   int sm_count = 0;
   std::atomic<unsigned> next_work_slot{0};   // round robin over the kernels' work counters
   bool ok = false;          // compute capability 10.0
-  bool fwd_attr[4] = {false, false, false, false};   // [HD 128, HD 64] x [whole ring, split]
-  bool bwd_attr = false;
+  // shared-memory attributes already set: [HD 128, HD 64] x [whole ring, split]; read and
+  // written by any host thread, hence atomic (setting an attribute twice is harmless)
+  std::atomic<bool> fwd_attr[4] = {false, false, false, false};
+  std::atomic<bool> bwd_attr{false};
 };
 
 std::mutex g_dev_mu;

@@ -100,6 +100,10 @@ def _stream(stream) -> int:
 def _need(t: torch.Tensor, name: str, dtype=None, shape=None) -> None:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    # the library launches on the current device (and uses its static scratch there)
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device} but the current device is cuda:{torch.cuda.current_device()}; "
+                         "make the tensors' device current (torch.cuda.device) before the call")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:

@@ -17,9 +17,15 @@ Causal masking is on global positions: block j is entirely visible to block r wh
 per element when j == r (the kernel's own causal mask, same positions), and skipped when j > r.
 The skipped blocks still travel on, so every rank forwards D - 1 blocks.
 
+Forward memory: each step's partial is folded into a running (o, lse) as soon as it is computed
+(_RunningMerge), so a rank holds two partials at most, whatever D -- the fixed per-host memory of
+§3.4 -- rather than one per ring step.
+
 Backward: rank r keeps dQ for its queries; the dK/dV accumulators (fp32) of a key/value block
 travel with that block, collect every rank's contribution, and are back at the block's owner
 after D hops.  The per-block backward uses the global O and lse, so each contribution is exact.
+K and V do not change during a step, so their transfer to the next rank is posted before the
+step's compute (overlapping it, §3.3); the accumulators follow once the step has added to them.
 
 Zig-zag assignment (ring_fwd_zigzag / ring_bwd_zigzag; the striped/zig-zag variant that the
 "Ring Attention" pages name as a follow-up): with contiguous blocks and a causal mask, rank r has
@@ -68,6 +74,88 @@ def _cuda_merge(o_parts, lse_parts):
     return ra.merge(o_parts, lse_parts, out_dtype=torch.bfloat16)
 
 
+def _cuda_merge_f32(o_parts, lse_parts):
+    from . import ring_attn as ra
+    return ra.merge(o_parts, lse_parts, out_dtype=torch.float32)
+
+
+def _raise_on_device_status():
+    """After a ring call on the CUDA library: synchronise and raise if a kernel gave up on a
+    bounded wait (its result would be incomplete).  One synchronisation per ring call."""
+    from . import ring_attn as ra
+    code = ra.device_status()
+    if code != ra.RA_OK:
+        raise ra.RingAttnError(code, "ring kernel")
+
+
+class _RunningMerge:
+    """The running log-sum-exp fold of one query block's per-step partials ("精读笔记 ...",
+    §3.1: blocks combined in any order through their statistics).  Each new partial is merged
+    into the running (o, lse) at once, so a rank holds at most two partials whatever the ring
+    length -- the fixed per-host memory of §3.4 -- instead of one per ring step.
+
+    Default (block_fwd and merge None): the CUDA library.  Each partial is written by
+    ring_attn_fwd_partial into slot 1 of a preallocated float32 pair [2][B, H, c, Dh] whose
+    slot 0 holds the running result; ring_attn_merge_ex folds the pair into slot 0 of a second
+    pair (float32, nothing rounded before the end), and the two pairs swap roles.  result()
+    rounds once, to the input dtype.  With callables: the same fold through `merge` on two
+    stacked parts (the caller's precision)."""
+
+    def __init__(self, q, block_fwd: Optional[BlockFwd], merge: Optional[Merge]):
+        self.cuda = block_fwd is None and merge is None
+        self.block_fwd = block_fwd or _cuda_block_fwd
+        self.merge = merge or _cuda_merge_f32     # running folds: nothing rounded yet
+        self.final = merge or _cuda_merge         # the last one rounds to the output dtype
+        self.state = None
+        self.held = 0          # partials (running result included) alive in the fold
+        self.peak = 0
+        if self.cuda:
+            B, H, c, Dh = q.shape
+            self.pairs = [torch.empty((2, B, H, c, Dh), dtype=torch.float32, device=q.device) for _ in range(2)]
+            self.lses = [torch.empty((2, B, H, c), dtype=torch.float32, device=q.device) for _ in range(2)]
+            self.n = 0
+
+    def _note(self, n):
+        self.held = n
+        self.peak = max(self.peak, n)
+
+    def add(self, q, k, v, masked):
+        if self.cuda:
+            from . import ring_attn as ra
+            a, la = self.pairs[0], self.lses[0]
+            slot = 0 if self.n == 0 else 1
+            ra.fwd_partial(q, k, v, 1, masked, out=a[slot], lse=la[slot])
+            self._note(slot + 1)
+            if self.n > 0:
+                ra.merge(a, la, out_dtype=torch.float32, out=self.pairs[1][0], lse=self.lses[1][0])
+                self.pairs.reverse()
+                self.lses.reverse()
+                self._note(1)
+            self.n += 1
+            return
+        o_t, l_t = self.block_fwd(q, k, v, masked)
+        if self.state is None:
+            self.state = (o_t, l_t)
+            self._note(1)
+            return
+        self._note(2)
+        o_r, l_r = self.state
+        self.state = self.merge(torch.stack((o_r.to(o_t.dtype), o_t)).contiguous(),
+                                torch.stack((l_r.to(l_t.dtype), l_t)).contiguous())
+        self._note(1)
+
+    def result(self, dtype):
+        if self.cuda:
+            from . import ring_attn as ra
+            if self.n == 0:
+                raise ValueError("no partial was added")
+            return ra.merge(self.pairs[0][:1], self.lses[0][:1], out_dtype=dtype)
+        if self.state is None:
+            raise ValueError("no partial was added")
+        o, l = self.state
+        return self.final(o.unsqueeze(0).contiguous(), l.unsqueeze(0).contiguous())
+
+
 def ring_steps(rank: int, world: int, causal: bool):
     """The blocks rank `rank` works on, in ring order: (step t, key/value block j, mask) for
     t = 0..world-1 with j = (rank - t) mod world; causal drops j > rank (nothing visible) and
@@ -94,10 +182,13 @@ class _Ring:
         return dist.get_global_rank(self.group, r) if self.group is not None else r
 
     def start(self, sends, recvs):
+        """Post the sends to rank + 1 and the receives from rank - 1; requests accumulate
+        until wait().  Every rank posts the same sequence of start() calls, so the batches
+        pair up in order."""
         nxt, prv = self._global((self.rank + 1) % self.world), self._global((self.rank - 1) % self.world)
         ops = [dist.P2POp(dist.isend, s, nxt, self.group) for s in sends]
         ops += [dist.P2POp(dist.irecv, r, prv, self.group) for r in recvs]
-        self._reqs = dist.batch_isend_irecv(ops)
+        self._reqs += dist.batch_isend_irecv(ops)
 
     def wait(self):
         for r in self._reqs:
@@ -106,29 +197,33 @@ class _Ring:
 
 
 def ring_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, group=None,
-             block_fwd: Optional[BlockFwd] = None, merge: Optional[Merge] = None
+             block_fwd: Optional[BlockFwd] = None, merge: Optional[Merge] = None, stats: Optional[dict] = None
              ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Forward of this rank's query block.  q, k, v: [B, H, c, Dh], this rank's block of the
-    sequence (rank r holds positions [r c, r c + c)).  Returns (o [B, H, c, Dh], lse [B, H, c])."""
+    sequence (rank r holds positions [r c, r c + c)).  Returns (o [B, H, c, Dh], lse [B, H, c]).
+    Each step's partial is folded into a running result at once (_RunningMerge), so the memory
+    a rank holds does not grow with the ring length.  `stats`, if given, receives
+    "peak_partials": the most partials held at once."""
     ring = _Ring(group)
-    block_fwd = block_fwd or _cuda_block_fwd
-    merge = merge or _cuda_merge
+    run = _RunningMerge(q, block_fwd, merge)
     kv = torch.stack((k, v)).contiguous()
     nxt = torch.empty_like(kv)
-    parts_o, parts_l = [], []
     work = {t: masked for t, _, masked in ring_steps(ring.rank, ring.world, causal)}
     for t in range(ring.world):
         more = t + 1 < ring.world
         if more:   # the next block is in flight while this one is computed
             ring.start([kv], [nxt])
         if t in work:
-            o_t, l_t = block_fwd(q, kv[0], kv[1], work[t])
-            parts_o.append(o_t.float())
-            parts_l.append(l_t.float())
+            run.add(q, kv[0], kv[1], work[t])
         if more:
             ring.wait()
             kv, nxt = nxt, kv
-    return merge(torch.stack(parts_o).contiguous(), torch.stack(parts_l).contiguous())
+    out = run.result(q.dtype)
+    if stats is not None:
+        stats["peak_partials"] = run.peak
+    if run.cuda:
+        _raise_on_device_status()
+    return out
 
 
 def ring_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
@@ -144,13 +239,18 @@ def ring_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     dq = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
     work = {t: masked for t, _, masked in ring_steps(ring.rank, ring.world, causal)}
     for t in range(ring.world):
+        hop = ring.world > 1   # D hops in all: the accumulators end at their block's owner
+        if hop:   # K, V do not change during the step: their transfer overlaps the compute
+            ring.start([kv], [kv_n])
         if t in work:
             block_acc(q, kv[0], kv[1], o, lse, do, work[t], dq, g[0], g[1])
-        if ring.world > 1:   # D hops in all: the accumulators end at their block's owner
-            ring.start([kv, g], [kv_n, g_n])
+        if hop:   # the block's dK, dV accumulators leave once this step's share is in
+            ring.start([g], [g_n])
             ring.wait()
             kv, kv_n = kv_n, kv
             g, g_n = g_n, g
+    if block_bwd is None:
+        _raise_on_device_status()
     return dq.to(q.dtype), g[0].to(q.dtype), g[1].to(q.dtype)
 
 
@@ -159,14 +259,13 @@ def ring_fwd_emulated(q_blocks, k_blocks, v_blocks, causal: bool = True, block_f
     """All ranks of ring_fwd in one process, without communication: rank r's output from the
     same ring_steps schedule, the blocks taken from the lists.  For checking the block-pair
     work of a D-rank ring on one device."""
-    block_fwd = block_fwd or _cuda_block_fwd
-    merge = merge or _cuda_merge
     world = len(q_blocks)
     outs = []
     for r in range(world):
-        parts = [block_fwd(q_blocks[r], k_blocks[j], v_blocks[j], masked) for _, j, masked in ring_steps(r, world, causal)]
-        outs.append(merge(torch.stack([o.float() for o, _ in parts]).contiguous(),
-                          torch.stack([l.float() for _, l in parts]).contiguous()))
+        run = _RunningMerge(q_blocks[r], block_fwd, merge)
+        for _, j, masked in ring_steps(r, world, causal):
+            run.add(q_blocks[r], k_blocks[j], v_blocks[j], masked)
+        outs.append(run.result(q_blocks[r].dtype))
     return outs
 
 
@@ -242,35 +341,29 @@ def _kv_halves(k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
     return torch.stack([torch.stack(p) for p in zip(_halves(k), _halves(v))]).contiguous()
 
 
-def _merge_halves(parts, merge):
-    outs = [merge(torch.stack([o for o, _ in p]).contiguous(), torch.stack([l for _, l in p]).contiguous())
-            for p in parts]
-    return torch.cat([o for o, _ in outs], dim=2), torch.cat([l for _, l in outs], dim=2)
-
-
 def ring_fwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, group=None,
                     block_fwd: Optional[BlockFwd] = None, merge: Optional[Merge] = None
                     ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Forward of this rank's zig-zag shard.  q, k, v: [B, H, c, Dh], zigzag_shard of the full
     sequence for this rank (c = S / world, even).  Returns (o, lse) in the same shard layout."""
     ring = _Ring(group)
-    block_fwd = block_fwd or _cuda_block_fwd
-    merge = merge or _cuda_merge
     qh = _halves(q)
+    runs = [_RunningMerge(h, block_fwd, merge) for h in qh]   # one running fold per query half
     kv = _kv_halves(k, v)
     nxt = torch.empty_like(kv)
-    parts = ([], [])
     for t, _, pairs in zigzag_steps(ring.rank, ring.world, causal):
         more = t + 1 < ring.world
         if more:   # the next shard is in flight while this one is computed
             ring.start([kv], [nxt])
         for a, b, masked in pairs:
-            o_t, l_t = block_fwd(qh[a], kv[b, 0], kv[b, 1], masked)
-            parts[a].append((o_t.float(), l_t.float()))
+            runs[a].add(qh[a], kv[b, 0], kv[b, 1], masked)
         if more:
             ring.wait()
             kv, nxt = nxt, kv
-    return _merge_halves(parts, merge)
+    outs = [r.result(q.dtype) for r in runs]
+    if runs[0].cuda:
+        _raise_on_device_status()
+    return torch.cat([o for o, _ in outs], dim=2), torch.cat([l for _, l in outs], dim=2)
 
 
 def ring_bwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
@@ -286,13 +379,18 @@ def ring_bwd_zigzag(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.
     kv_n, g_n = torch.empty_like(kv), torch.empty_like(g)
     dq = [torch.zeros(h.shape, dtype=torch.float32, device=h.device) for h in qh]
     for t, _, pairs in zigzag_steps(ring.rank, ring.world, causal):
+        hop = ring.world > 1   # D hops in all: the accumulators end at their shard's owner
+        if hop:   # K, V do not change during the step: their transfer overlaps the compute
+            ring.start([kv], [kv_n])
         for a, b, masked in pairs:
             block_acc(qh[a], kv[b, 0], kv[b, 1], oh[a], lh[a], dh[a], masked, dq[a], g[b, 0], g[b, 1])
-        if ring.world > 1:   # D hops in all: the accumulators end at their shard's owner
-            ring.start([kv, g], [kv_n, g_n])
+        if hop:   # the halves' dK, dV accumulators leave once this step's share is in
+            ring.start([g], [g_n])
             ring.wait()
             kv, kv_n = kv_n, kv
             g, g_n = g_n, g
+    if block_bwd is None:
+        _raise_on_device_status()
     dt = q.dtype
     return (torch.cat(dq, dim=2).to(dt), torch.cat((g[0, 0], g[1, 0]), dim=2).to(dt),
             torch.cat((g[0, 1], g[1, 1]), dim=2).to(dt))
@@ -302,19 +400,17 @@ def ring_fwd_zigzag_emulated(q_shards, k_shards, v_shards, causal: bool = True,
                              block_fwd: Optional[BlockFwd] = None, merge: Optional[Merge] = None):
     """All ranks of ring_fwd_zigzag in one process, without communication: rank r's (o, lse)
     from the same zigzag_steps schedule, the shards taken from the lists."""
-    block_fwd = block_fwd or _cuda_block_fwd
-    merge = merge or _cuda_merge
     world = len(q_shards)
     kvs = [_kv_halves(k, v) for k, v in zip(k_shards, v_shards)]
     outs = []
     for r in range(world):
         qh = _halves(q_shards[r])
-        parts = ([], [])
+        runs = [_RunningMerge(h, block_fwd, merge) for h in qh]
         for _, j, pairs in zigzag_steps(r, world, causal):
             for a, b, masked in pairs:
-                o_t, l_t = block_fwd(qh[a], kvs[j][b, 0], kvs[j][b, 1], masked)
-                parts[a].append((o_t.float(), l_t.float()))
-        outs.append(_merge_halves(parts, merge))
+                runs[a].add(qh[a], kvs[j][b, 0], kvs[j][b, 1], masked)
+        res = [run.result(q_shards[r].dtype) for run in runs]
+        outs.append((torch.cat([o for o, _ in res], dim=2), torch.cat([l for _, l in res], dim=2)))
     return outs
 
 

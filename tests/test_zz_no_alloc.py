@@ -5,8 +5,9 @@ framework that owns every device allocation, or latency-critical code that canno
 cudaMalloc's implicit synchronisation -- so they cannot hand ring_attn_bwd its workspace.
 ring_attn_bwd_noalloc keeps that scratch in a static device array of the library instead.
 These tests call it through the C ABI and compare it with ring_attn_bwd (given a workspace)
-within the parity tolerances; consecutive calls check that leftovers in the shared scratch
-from the previous call do not leak into the next result.
+and with the float64 oracle, within the parity tolerances; consecutive calls check that
+leftovers in the shared scratch from the previous call do not leak into the next result, and
+that a call with caller-provided outputs allocates no device memory.
 
 This file is collected last on purpose, so a stop-at-first-failure run reaches it only
 after every other test has run.
@@ -16,6 +17,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from long_context_exact_fwd_b200.workloads import random_qkv
 from parity import assert_close_bf16
 
@@ -37,6 +39,10 @@ def _problem(ra, B, H, S, D, causal, seed):
     return q, k, v, o, lse, do
 
 
+def _oracle_grads(q, k, v, do, causal):
+    return oracle.attn_bwd_heads(*(x.cpu() for x in (q, k, v, do)), causal)
+
+
 def _compare(got, ref):
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
         assert_close_bf16(g.float().cpu().numpy(), r.float().cpu().numpy(), name)
@@ -46,11 +52,20 @@ def _compare(got, ref):
 def test_noalloc_matches_workspace_backward_on_consecutive_calls(ra, causal):
     q, k, v, o, lse, do = _problem(ra, 1, 2, 1000, 8, causal, seed=41)
     ref = ra.bwd(q, k, v, o, lse, do, 8, causal)
+    want = _oracle_grads(q, k, v, do, causal)
     torch.cuda.synchronize()
-    for _ in range(2):   # the second call starts from the first call's leftovers
-        got = ra.bwd_noalloc(q, k, v, o, lse, do, 8, causal)
+    outs = [torch.empty_like(q) for _ in range(3)]   # caller-owned outputs
+    for i in range(2):   # the second call starts from the first call's leftovers
+        if i == 1:
+            alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+        got = ra.bwd_noalloc(q, k, v, o, lse, do, 8, causal, *outs)
         assert ra.device_status() == 0
+        if i == 1:   # a warmed-up call allocates nothing, through torch or behind its back
+            assert torch.cuda.memory_allocated() == alloc0
+            assert torch.cuda.mem_get_info()[0] == free0
         _compare(got, ref)
+        for name, g, r in zip(("dq", "dk", "dv"), got, want):
+            assert_close_bf16(g.float().cpu().numpy(), r, name)
     # a different, smaller problem right after: nothing of the larger one may remain
     q2, k2, v2, o2, lse2, do2 = _problem(ra, 2, 1, 384, 3, causal, seed=43)
     ref2 = ra.bwd(q2, k2, v2, o2, lse2, do2, 3, causal)
