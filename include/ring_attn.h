@@ -70,7 +70,7 @@ typedef void* ra_stream;
  *            accumulated and rounded to nearest even once.
  *   lse      [B][H][S] float32, written: the row log-sum-exp (natural log).
  *   B, H, S  >= 1.  S need not be a multiple of the kernel's 128-row tiles.
- *   Dh       head dimension; 128 on this path (else RA_ERR_SHAPE).
+ *   Dh       head dimension: 64 or 128 (else RA_ERR_SHAPE).
  *   D        number of ring blocks, 1 <= D <= S and S % D == 0 (the pages' even split,
  *            "limitations" paragraph of the close reading), else RA_ERR_SHAPE.
  *   causal   0 or 1 (see Mask above).
@@ -158,15 +158,30 @@ RA_API size_t ring_attn_bwd_workspace_size(int B, int H, int S, int Dh);
  *   q, k, v, o, dO : [B][H][S][Dh] bf16, read only, 16-byte aligned (o from ring_attn_fwd).
  *   lse            : [B][H][S] float32 from ring_attn_fwd.
  *   dq, dk, dv     : [B][H][S][Dh] bf16, written (fully overwritten).
+ *   Dh             : 64 or 128 (else RA_ERR_SHAPE).
  *   workspace      : >= ring_attn_bwd_workspace_size(B, H, S, Dh) bytes of device memory,
  *                    256-byte aligned; its contents on entry are ignored (it is cleared
  *                    on the stream) and undefined on return.
  *   Other arguments as ring_attn_fwd.  Each key/value tile visits the query tiles that
- *   can see it, in ring order.
+ *   can see it, in ring order.  Three launches on `stream` (Delta preprocess, main kernel, dQ
+ *   conversion).  Errors: RA_ERR_ARG (null pointer, non-positive size), RA_ERR_SHAPE,
+ *   RA_ERR_ALIGN, RA_ERR_WORKSPACE (null, not 256-byte aligned or too small), RA_ERR_CUDA.
  */
 RA_API int ring_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                   void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D, int causal, void* workspace,
                   size_t workspace_bytes, ra_stream stream);
+
+/*
+ * ring_attn_bwd_ex -- ring_attn_bwd with an explicit softmax scale: the gradient of
+ * ring_attn_fwd_ex called with the same scale (page "精读笔记 ...", §4.2: training runs through
+ * the same blockwise ring; the scale enters P = exp(scale q k^T - lse), dQ = scale dS K and
+ * dK = scale dS^T Q).  scale > 0 overrides 1/sqrt(Dh); scale <= 0 (or not finite) keeps the
+ * default.  lse must come from a forward with the same scale.  Other arguments, launches and
+ * errors as ring_attn_bwd.
+ */
+RA_API int ring_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dO, void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D,
+                            int causal, float scale, void* workspace, size_t workspace_bytes, ra_stream stream);
 
 /*
  * ring_attn_bwd_accumulate -- ring_attn_bwd whose gradients are added, in float32, to the
@@ -176,7 +191,7 @@ RA_API int ring_attn_bwd(const void* q, const void* k, const void* v, const void
  * §4.2: training runs through the same blockwise ring), rounded once by the caller at the end.
  *   q, k, v, o, lse, dO, B, H, S, Dh, D, causal, workspace  as ring_attn_bwd.
  *   dq32, dk32, dv32  [B][H][S][Dh] float32, 16-byte aligned, read and written; the caller
- *                     clears them before the first call.
+ *                     clears them before the first call.  Dh 64 or 128.
  * Launches as ring_attn_bwd, with the last one adding the scaled dQ instead of converting it.
  * Errors as ring_attn_bwd.
  */
@@ -191,8 +206,9 @@ RA_API int ring_attn_bwd_accumulate(const void* q, const void* k, const void* v,
  * cudaMalloc (or any allocator) on their path -- for example code embedded in a host
  * framework that owns every device allocation, or latency-critical code that cannot afford
  * cudaMalloc's implicit synchronisation -- and so cannot supply ring_attn_bwd's workspace.
- *   Arguments are those of ring_attn_bwd without the workspace.  The fp32 dQ accumulator and
- *   the per-row statistics live instead in one static device array of the library of
+ *   Arguments are those of ring_attn_bwd without the workspace (Dh 64 or 128).  The fp32 dQ
+ *   accumulator and the per-row statistics live instead in one static device array of the
+ *   library of
  *   ring_attn_bwd_noalloc_max_bytes() bytes (96 MiB), reserved on every device that loads the
  *   library until the process exits.  A problem whose ring_attn_bwd_workspace_size exceeds that
  *   size is rejected with RA_ERR_WORKSPACE before anything is enqueued.

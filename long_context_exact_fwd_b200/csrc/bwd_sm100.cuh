@@ -18,25 +18,28 @@
 //               the fp32 accumulator by TMA bulk reduce-add.
 //   bwd_convert dQ = scale * accumulator -> bf16 (HBM-bound).
 //
-// bwd_kernel CTA (512 threads):
+// bwd_kernel<HD> CTA (512 threads; head dimension HD = 64 or 128):
 //   warpgroups 0, 1  thread = key row, warpgroup h taking query columns [64h, 64h + 64): P^T,
 //                dS^T (bf16) into TMEM and dS into shared memory; final dK, dV epilogue (head
-//                columns [64h, 64h + 64)).  Each writes TMEM only inside columns it has itself
-//                read, so the two never race.
-//   warpgroup 2  thread = query row: reads dQ from TMEM, stages it (fp32, four 128-B swizzled
-//                32-column boxes, 64 KB) over the query tile's own Q/dO stage once dK has read
-//                Q, and one thread issues the TMA reduce-adds into the fp32 accumulator and
-//                then hands the stage back to the producer.
+//                columns [HD/2 h, HD/2 (h + 1))).  Each writes TMEM only inside columns it has
+//                itself read, so the two never race.
+//   warpgroup 2  thread = query row: reads dQ from TMEM, stages it (fp32, HD/32 128-B swizzled
+//                boxes of 32 columns x 128 rows) over the query tile's own Q/dO stage once dK
+//                has read Q, and one thread issues the TMA reduce-adds into the fp32
+//                accumulator and then hands the stage back to the producer.
 //   warp 12      TMA producer: K, V once per item; Q, dO, lse2, Delta per query tile (2 stages).
 //   warp 13      TMEM allocator + tcgen05.mma issuer (warps 14, 15 complete warpgroup 3).
 // TMEM (512 columns): [0,128) S^T, then P^T (bf16) of queries 0-63 in [0,32) and of queries
-//   64-127 in [96,128); [128,256) dP^T, then dS^T in [128,160) and [224,256), then dQ once
-//   dK has consumed dS^T; [256,384) dV; [384,512) dK.
-// MMAs per query tile (M = N = K = 128 each, in this order): S^T = K Q^T, dP^T = V dO^T,
-//   dV += P^T dO, dK += dS^T Q, dQ = dS K.  The tensor pipe executes them in issue order, so
-//   a later MMA may overwrite TMEM an earlier one reads: S^T of the next tile is issued right
-//   after dQ (P^T is dead once dV issued), and only its dP^T waits for the dQ readout.
+//   64-127 in [96,128); [128,256) dP^T, then dS^T in [128,160) and [224,256), then dQ (HD
+//   columns) once dK has consumed dS^T; [256, 256 + HD) dV; [256 + HD, 256 + 2 HD) dK.
+// MMAs per query tile (M = 128; in this order): S^T = K Q^T (N = 128, K = HD), dP^T = V dO^T,
+//   dV += P^T dO (N = HD, K = 128), dK += dS^T Q, dQ = dS K (N = HD, K = 128).  The tensor
+//   pipe executes them in issue order, so a later MMA may overwrite TMEM an earlier one reads:
+//   S^T of the next tile is issued right after dQ (P^T is dead once dV issued), and only its
+//   dP^T waits for the dQ readout.
 #pragma once
+#include <type_traits>
+
 #include "ra_schedule.h"
 #include "ra_sm100.cuh"
 #include "ra_work.cuh"
@@ -46,7 +49,6 @@ namespace bwd {
 
 constexpr int BM = 128;   // keys per CTA tile (TMEM lanes of S^T, dP^T, dV, dK)
 constexpr int BQ = 128;   // queries per query tile
-constexpr int HD = 128;   // head dimension of this kernel
 constexpr int NSTAGE = 2;
 constexpr int NUM_THREADS = 512;
 constexpr int WARP_TMA = 12, WARP_MMA = 13;
@@ -72,18 +74,24 @@ constexpr uint32_t TMEM_COLS = 512;
 #ifndef RA_BWD_EXP2_FMA_PER4
 #define RA_BWD_EXP2_FMA_PER4 0
 #endif
-constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 384;
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256;
+template <int HD>
+__host__ __device__ constexpr uint32_t col_dk() { return COL_DV + HD; }
 // bf16 P^T / dS^T of query columns [64h, 64h + 64): TMEM columns [base, base + 32)
 __host__ __device__ constexpr uint32_t col_p(int h) { return h ? 96u : 0u; }
 __host__ __device__ constexpr uint32_t col_ds(int h) { return h ? 224u : 128u; }
 
+template <int HD>
 struct Layout {
+  static_assert(HD == 64 || HD == 128, "head dim");
+  static constexpr int SUB = HD / 64;                  // 128-byte-swizzled column blocks of a tile
   static constexpr int SUB_BYTES = 128 * 128;          // 128 rows x 128 B (64 bf16)
-  static constexpr int TILE_BYTES = 2 * SUB_BYTES;     // 128 rows x 128 bf16
+  static constexpr int TILE_BYTES = SUB * SUB_BYTES;   // 128 rows x HD bf16
+  static constexpr int DS_BYTES = 2 * SUB_BYTES;       // 128 keys x 128 queries bf16
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE_BYTES;
   static constexpr int DS_OFF = V_OFF + TILE_BYTES;    // dS, MN-major: two 64-query halves
-  static constexpr int STAGE_OFF = DS_OFF + TILE_BYTES;
+  static constexpr int STAGE_OFF = DS_OFF + DS_BYTES;
   static constexpr int STAGE_Q = 0, STAGE_DO = TILE_BYTES, STAGE_LSE = 2 * TILE_BYTES,
                        STAGE_DELTA = STAGE_LSE + BQ * 4, STAGE_BYTES = STAGE_DELTA + BQ * 4;
   static constexpr int BAR_OFF = STAGE_OFF + NSTAGE * STAGE_BYTES;
@@ -95,8 +103,11 @@ struct Layout {
   static constexpr uint32_t WQ_CONSUMERS = 1 + 12;   // MMA thread + one arrival per warp of warpgroups 0-2
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, item ring[2]
   static constexpr int BYTES = MISC_OFF + 16;
+  // the dQ staging (HD/32 boxes of 128 rows x 128 B) fits over a stage's Q and dO tiles
+  static_assert((HD / 32) * SUB_BYTES <= 2 * TILE_BYTES, "dQ staging");
+  static_assert(STAGE_BYTES % 1024 == 0 && STAGE_OFF % 1024 == 0, "swizzled tiles need 1024-B alignment");
 };
-static_assert(Layout::BYTES <= 232448, "shared memory");
+static_assert(Layout<128>::BYTES <= 232448 && Layout<64>::BYTES <= 232448, "shared memory");
 
 struct Params {
   int BH, S, S_pad, D, causal;
@@ -137,10 +148,11 @@ __device__ __forceinline__ void advance(int& stage, uint32_t& phase) {
 }
 
 // ------------------------------------------------------------------ producer
+template <int HD>
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const CUtensorMap* tm_do, const Params& p, uint32_t sbase, volatile int* wq,
                          volatile int* abort_flag) {
-  using L = Layout;
+  using L = Layout<HD>;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
@@ -156,7 +168,7 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
     item_coords(w, p, bh, kt);
     if (!mbar_wait(bar(L::B_KV_EMPTY), kv_phase ^ 1u, abort_flag)) { ok = false; break; }
     mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * L::TILE_BYTES);
-    for (int sb = 0; sb < 2; ++sb) {
+    for (int sb = 0; sb < L::SUB; ++sb) {
       tma_load_3d(tm_k, sbase + L::K_OFF + sb * L::SUB_BYTES, bar(L::B_KV_FULL), sb * 64, kt * BM, bh);
       tma_load_3d(tm_v, sbase + L::V_OFF + sb * L::SUB_BYTES, bar(L::B_KV_FULL), sb * 64, kt * BM, bh);
     }
@@ -170,7 +182,7 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
       const uint32_t full = bar(L::B_QD_FULL + stage);
       const uint32_t st = sbase + L::STAGE_OFF + stage * L::STAGE_BYTES;
       mbar_arrive_expect_tx(full, 2 * L::TILE_BYTES + 2 * BQ * 4);
-      for (int sb = 0; sb < 2; ++sb) {
+      for (int sb = 0; sb < L::SUB; ++sb) {
         tma_load_3d(tm_q, st + L::STAGE_Q + sb * L::SUB_BYTES, full, sb * 64, qt * BQ, bh);
         tma_load_3d(tm_do, st + L::STAGE_DO + sb * L::SUB_BYTES, full, sb * 64, qt * BQ, bh);
       }
@@ -193,40 +205,44 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
 }
 
 // ------------------------------------------------------------------ MMA issuer
+template <int HD>
 __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, bool first_zero) {
-  // D[128 x 128] = A[128 x 128] * B[128 x 128]^T, both K-major 128-B swizzled (two 64-col halves)
+  // D[128 x 128] = A[128 x HD] * B[128 x HD]^T, both K-major 128-B swizzled (64-column blocks)
   constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * Layout::SUB_BYTES + (kk & 3) * 32;
+    const uint32_t off = (kk >> 2) * Layout<HD>::SUB_BYTES + (kk & 3) * 32;
     umma_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), IDESC,
             (first_zero && kk == 0) ? 0u : 1u);
   }
 }
 
+template <int HD>
 __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_smem,
                                            bool accumulate) {
-  // D[128 x 128] (+)= A[128 x 128] (TMEM, bf16; K = 0-63 at a_lo, 64-127 at a_hi)
-  //                   * B[128 x 128] (smem, MN-major: rows = K)
+  // D[128 x HD] (+)= A[128 x 128] (TMEM, bf16; K = 0-63 at a_lo, 64-127 at a_hi)
+  //                  * B[128 x HD] (smem, MN-major: rows = K, 64-column blocks SUB_BYTES apart)
   constexpr uint32_t IDESC = idesc_bf16_f32(128, HD, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < BQ / 16; ++kk)
-    umma_ts(d_tmem, (kk < 4 ? a_lo : a_hi) + (kk & 3) * 8, sdesc_sw128(b_smem + kk * 2048, Layout::SUB_BYTES, 1024),
-            IDESC, (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, (kk < 4 ? a_lo : a_hi) + (kk & 3) * 8,
+            sdesc_sw128(b_smem + kk * 2048, Layout<HD>::SUB_BYTES, 1024), IDESC, (accumulate || kk > 0) ? 1u : 0u);
 }
 
+template <int HD>
 __device__ __forceinline__ void mma_dq(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_smem) {
-  // dQ [128 q x 128] = dS [128 q x 128 k] (MN-major: q contiguous, two 64-q halves)
-  //                   * K [128 k x 128] (MN-major: rows = K, two 64-column halves)
+  // dQ [128 q x HD] = dS [128 q x 128 k] (MN-major: q contiguous, two 64-q halves)
+  //                  * K [128 k x HD] (MN-major: rows = K, 64-column blocks)
   constexpr uint32_t IDESC = idesc_bf16_f32(128, HD, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < BM / 16; ++kk)
-    umma_ss(d_tmem, sdesc_sw128(ds_smem + kk * 2048, Layout::SUB_BYTES, 1024),
-            sdesc_sw128(k_smem + kk * 2048, Layout::SUB_BYTES, 1024), IDESC, kk > 0 ? 1u : 0u);
+    umma_ss(d_tmem, sdesc_sw128(ds_smem + kk * 2048, Layout<HD>::SUB_BYTES, 1024),
+            sdesc_sw128(k_smem + kk * 2048, Layout<HD>::SUB_BYTES, 1024), IDESC, kk > 0 ? 1u : 0u);
 }
 
+template <int HD>
 __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
-  using L = Layout;
+  using L = Layout<HD>;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0, p_phase = 0, ds_phase = 0, dqf_phase = 0;
@@ -251,25 +267,25 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
       if (!mbar_wait(bar(L::B_QD_FULL + s), phase, abort_flag)) { ok = false; break; }
       advance(stage, phase);
       tc_fence_after();
-      mma_kmajor(tmem + COL_S, sbase + L::K_OFF, st + L::STAGE_Q, true);     // S^T = K Q^T
+      mma_kmajor<HD>(tmem + COL_S, sbase + L::K_OFF, st + L::STAGE_Q, true);     // S^T = K Q^T
       tc_commit(bar(L::B_S_FULL));
       if (dq_pending) {  // dP^T overwrites the columns the previous tile's dQ readout reads
         if (!mbar_wait(bar(L::B_DQ_FREE), dqf_phase, abort_flag)) { ok = false; break; }
         dqf_phase ^= 1u;
         tc_fence_after();
       }
-      mma_kmajor(tmem + COL_DP, sbase + L::V_OFF, st + L::STAGE_DO, true);   // dP^T = V dO^T
+      mma_kmajor<HD>(tmem + COL_DP, sbase + L::V_OFF, st + L::STAGE_DO, true);   // dP^T = V dO^T
       tc_commit(bar(L::B_DP_FULL));
       if (!mbar_wait(bar(L::B_P_READY), p_phase, abort_flag)) { ok = false; break; }
       p_phase ^= 1u;
       tc_fence_after();
-      mma_tmem_a(tmem + COL_DV, tmem + col_p(0), tmem + col_p(1), st + L::STAGE_DO, n > 0);   // dV += P^T dO
+      mma_tmem_a<HD>(tmem + COL_DV, tmem + col_p(0), tmem + col_p(1), st + L::STAGE_DO, n > 0);   // dV += P^T dO
       if (!mbar_wait(bar(L::B_DS_READY), ds_phase, abort_flag)) { ok = false; break; }
       ds_phase ^= 1u;
       tc_fence_after();
-      mma_tmem_a(tmem + COL_DK, tmem + col_ds(0), tmem + col_ds(1), st + L::STAGE_Q, n > 0);   // dK += dS^T Q
+      mma_tmem_a<HD>(tmem + col_dk<HD>(), tmem + col_ds(0), tmem + col_ds(1), st + L::STAGE_Q, n > 0);   // dK += dS^T Q
       tc_commit(bar(L::B_DK_DONE));   // Q and dO of this stage no longer read by the tensor core
-      mma_dq(tmem + COL_DQ, sbase + L::DS_OFF, sbase + L::K_OFF);                 // dQ = dS K
+      mma_dq<HD>(tmem + COL_DQ, sbase + L::DS_OFF, sbase + L::K_OFF);                 // dQ = dS K
       tc_commit(bar(L::B_DQ_FULL));
       dq_pending = true;
     }
@@ -282,10 +298,10 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
 }
 
 // ------------------------------------------------------------------ warpgroups 0, 1: P^T, dS^T, epilogue
-template <int half>
+template <int HD, int half>
 __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint32_t tmem, volatile int* wq,
                             volatile int* abort_flag) {
-  using L = Layout;
+  using L = Layout<HD>;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   const int lane = threadIdx.x & 31;
   const int quarter = (threadIdx.x >> 5) & 3;
@@ -404,19 +420,20 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
       tc_fence_before();
       mbar_arrive(bar(L::B_DS_READY));
     }
-    // ---- epilogue: dV, dK (scaled), head columns [64 half, 64 half + 64)
+    // ---- epilogue: dV, dK (scaled), head columns [HD/2 half, HD/2 (half + 1))
     if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC_FULL), acc_phase, abort_flag))) return;
     acc_phase ^= 1u;
     tc_fence_after();
+    constexpr int hc0 = (HD / 2) * half;   // this warpgroup's first head column
     const bool row_ok = k_row < p.S;
-    const size_t off = (static_cast<size_t>(bh) * p.S + k_row) * HD + qc0;
+    const size_t off = (static_cast<size_t>(bh) * p.S + k_row) * HD + hc0;
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
-      const uint32_t col = (which ? COL_DK : COL_DV) + qc0;
+      const uint32_t col = (which ? col_dk<HD>() : COL_DV) + hc0;
       const float mul = which ? p.scale : 1.f;
       __nv_bfloat16* dst_row = (which ? p.dk : p.dv) + off;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < HD / 64; ++c) {
         uint32_t rr[32];
         tmem_ld32(lane_base + col + 32 * c, rr);
         tmem_ld_wait();
@@ -450,9 +467,10 @@ __device__ void key_rows_wg(const Params& p, uint8_t* smem, uint32_t sbase, uint
 }
 
 // ------------------------------------------------------------------ warpgroup 2: dQ readout
+template <int HD>
 __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t* smem, uint32_t sbase, uint32_t tmem,
                               volatile int* wq, volatile int* abort_flag) {
-  using L = Layout;
+  using L = Layout<HD>;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   const int lane = threadIdx.x & 31;
   const int quarter = (threadIdx.x >> 5) & 3;
@@ -482,7 +500,7 @@ __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t
       tc_fence_after();
       uint32_t r[HD];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + COL_DQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      for (int c = 0; c < HD / 32; ++c) tmem_ld32(lane_base + COL_DQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar(L::B_DQ_FREE));   // dQ is in registers: hand the TMEM columns back
@@ -495,10 +513,10 @@ __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t
         stage = 0;
         qphase ^= 1u;
       }
-      // dQ row -> four 32-column fp32 boxes (128 B per row, 128-B swizzle) over Q and dO
+      // dQ row -> HD/32 32-column fp32 boxes (128 B per row, 128-B swizzle) over Q and dO
       uint8_t* st_row = smem + L::STAGE_OFF + s_idx * L::STAGE_BYTES + row * 128;
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
+      for (int b = 0; b < HD / 32; ++b)
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           *reinterpret_cast<uint4*>(st_row + b * L::SUB_BYTES + ((j ^ sw) << 4)) =
@@ -508,7 +526,7 @@ __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t
       if (leader) {
         const uint32_t st = sbase + L::STAGE_OFF + s_idx * L::STAGE_BYTES;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tma_reduce_add_3d(tm_dq, st + b * L::SUB_BYTES, 32 * b, qt * BQ, bh);
+        for (int b = 0; b < HD / 32; ++b) tma_reduce_add_3d(tm_dq, st + b * L::SUB_BYTES, 32 * b, qt * BQ, bh);
         bulk_commit();
         bulk_wait_read_all();
         mbar_arrive(bar(L::B_QD_EMPTY + s_idx));   // the producer may refill this stage
@@ -520,11 +538,12 @@ __device__ void query_rows_wg(const Params& p, const CUtensorMap* tm_dq, uint8_t
 }
 
 // ------------------------------------------------------------------ main kernel
+template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dq, const Params p) {
-  using L = Layout;
+  using L = Layout<HD>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
@@ -564,21 +583,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp >= 12) {
     regs_lower<REGS_OTHER>();
     if (warp == WARP_TMA) {
-      if ((threadIdx.x & 31) == 0) producer(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, wq, abort_flag);
+      if ((threadIdx.x & 31) == 0) producer<HD>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, wq, abort_flag);
       __syncwarp();
     } else if (warp == WARP_MMA) {
-      if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, wq, abort_flag);
+      if ((threadIdx.x & 31) == 0) mma_issuer<HD>(p, sbase, tmem, wq, abort_flag);
       __syncwarp();
     }
   } else if (warp < 8) {
     regs_raise<REGS_KEYS>();
     if (warp < 4)
-      key_rows_wg<0>(p, smem, sbase, tmem, wq, abort_flag);
+      key_rows_wg<HD, 0>(p, smem, sbase, tmem, wq, abort_flag);
     else
-      key_rows_wg<1>(p, smem, sbase, tmem, wq, abort_flag);
+      key_rows_wg<HD, 1>(p, smem, sbase, tmem, wq, abort_flag);
   } else {
     regs_raise<REGS_DQ>();
-    query_rows_wg(p, &tm_dq, smem, sbase, tmem, wq, abort_flag);
+    query_rows_wg<HD>(p, &tm_dq, smem, sbase, tmem, wq, abort_flag);
   }
 
   tc_fence_before();
@@ -593,7 +612,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 constexpr int PRE_WARPS = 8;
 
 // One warp per padded row: -Delta = -sum_d dO * O and -lse * log2(e) (0 and -inf in the
-// padding rows), and the row of the fp32 dQ accumulator cleared.
+// padding rows), and the row of the fp32 dQ accumulator cleared.  HD / 32 values per lane.
+template <int HD>
 __global__ void __launch_bounds__(PRE_WARPS * 32)
     bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                    const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
@@ -611,21 +631,25 @@ __global__ void __launch_bounds__(PRE_WARPS * 32)
     return;
   }
   const long long row = bh * S + s;
-  // HD = 128 bf16 per row: 8 bytes (4 values) per lane
-  const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + row * HD) + lane);
-  const uint2 b = __ldg(reinterpret_cast<const uint2*>(dO + row * HD) + lane);
+  constexpr int PER_LANE = HD / 32;   // bf16 values of a row per lane: 4 (8 bytes) or 2 (4 bytes)
+  using Vec = typename std::conditional<PER_LANE == 4, uint2, uint32_t>::type;
+  const Vec a = __ldg(reinterpret_cast<const Vec*>(o + row * HD) + lane);
+  const Vec b = __ldg(reinterpret_cast<const Vec*>(dO + row * HD) + lane);
   const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
   const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
   float acc = 0.f;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < PER_LANE / 2; ++i) {
     const float2 fa = __bfloat1622float2(a2[i]), fb = __bfloat1622float2(b2[i]);
     acc = fmaf(fa.x, fb.x, acc);
     acc = fmaf(fa.y, fb.y, acc);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  reinterpret_cast<float4*>(dq_acc + row * HD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if constexpr (PER_LANE == 4)
+    reinterpret_cast<float4*>(dq_acc + row * HD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+  else
+    reinterpret_cast<float2*>(dq_acc + row * HD)[lane] = make_float2(0.f, 0.f);
   if (lane == 0) {
     delta[prow] = -acc;
     lse2[prow] = -lse[row] * 1.4426950408889634f;

@@ -59,7 +59,7 @@ struct DevInfo {
   // shared-memory attributes already set: [HD 128, HD 64] x [whole ring, split]; read and
   // written by any host thread, hence atomic (setting an attribute twice is harmless)
   std::atomic<bool> fwd_attr[4] = {false, false, false, false};
-  std::atomic<bool> bwd_attr{false};
+  std::atomic<bool> bwd_attr[2] = {false, false};   // [HD 128, HD 64]
 };
 
 std::mutex g_dev_mu;
@@ -228,6 +228,7 @@ BwdWorkspace bwd_workspace(long long BH, int S, int Dh) {
 
 // dq32 given: dQ, dK, dV are added to the fp32 dq32, dk32, dv32 instead of written to the
 // bf16 dq, dk, dv.
+template <int HD>
 int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
              void* dk, void* dv, int B, int H, int S, int D, int causal, float scale, void* workspace,
              cudaStream_t stream, float* dq32 = nullptr, float* dk32 = nullptr, float* dv32 = nullptr) {
@@ -236,7 +237,7 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   DevInfo* di = dev_info(&st);
   if (!di) return st;
   const long long BH = static_cast<long long>(B) * H;
-  const BwdWorkspace ws = bwd_workspace(BH, S, rb::HD);
+  const BwdWorkspace ws = bwd_workspace(BH, S, HD);
   const int S_pad = (S + 127) / 128 * 128;
   float* dq_acc = static_cast<float*>(workspace);
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.dq_bytes);
@@ -246,19 +247,19 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   const long long prow = BH * S_pad;
   const long long pre_blocks = (prow + rb::PRE_WARPS - 1) / rb::PRE_WARPS;
   if (pre_blocks > INT_MAX) return RA_ERR_SHAPE;
-  rb::bwd_pre_kernel<<<static_cast<int>(pre_blocks), rb::PRE_WARPS * 32, 0, stream>>>(
+  rb::bwd_pre_kernel<HD><<<static_cast<int>(pre_blocks), rb::PRE_WARPS * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, delta, lse2, dq_acc,
       static_cast<int>(BH), S, S_pad);
   if ((st = launch_status()) != RA_OK) return st;
 
   // 2. key/value-stationary main kernel
   CUtensorMap mq, mk, mv, mdo;
-  if ((st = make_map(&mq, q, BH, S, rb::HD, rb::BQ)) != RA_OK) return st;
-  if ((st = make_map(&mk, k, BH, S, rb::HD, rb::BM)) != RA_OK) return st;
-  if ((st = make_map(&mv, v, BH, S, rb::HD, rb::BM)) != RA_OK) return st;
-  if ((st = make_map(&mdo, dO, BH, S, rb::HD, rb::BQ)) != RA_OK) return st;
+  if ((st = make_map(&mq, q, BH, S, HD, rb::BQ)) != RA_OK) return st;
+  if ((st = make_map(&mk, k, BH, S, HD, rb::BM)) != RA_OK) return st;
+  if ((st = make_map(&mv, v, BH, S, HD, rb::BM)) != RA_OK) return st;
+  if ((st = make_map(&mdo, dO, BH, S, HD, rb::BQ)) != RA_OK) return st;
   CUtensorMap mdq;   // fp32 accumulator, 32-column boxes for the reduce-adds
-  if ((st = make_map(&mdq, dq_acc, BH, S, rb::HD, rb::BQ, true)) != RA_OK) return st;
+  if ((st = make_map(&mdq, dq_acc, BH, S, HD, rb::BQ, true)) != RA_OK) return st;
   rb::Params p;
   p.BH = static_cast<int>(BH);
   p.S = S;
@@ -269,7 +270,7 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   const long long items = BH * p.n_kt;
   if (items > INT_MAX) return RA_ERR_SHAPE;
   p.n_items = static_cast<int>(items);
-  p.hgroup = heads_per_l2_group(BH, 4ll * S * rb::HD);   // Q + dO bytes of one head
+  p.hgroup = heads_per_l2_group(BH, 4ll * S * HD);   // Q + dO bytes of one head
   p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -280,25 +281,26 @@ int bwd_bf16(const void* q, const void* k, const void* v, const void* o, const f
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.dk32 = dq32 ? dk32 : nullptr;
   p.dv32 = dq32 ? dv32 : nullptr;
-  constexpr int smem = rb::Layout::BYTES;
-  if (!di->bwd_attr) {
-    const cudaError_t e = cudaFuncSetAttribute(rb::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr int smem = rb::Layout<HD>::BYTES;
+  constexpr int aslot = HD == 128 ? 0 : 1;
+  if (!di->bwd_attr[aslot]) {
+    const cudaError_t e = cudaFuncSetAttribute(rb::bwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(bwd smem)");
-    di->bwd_attr = true;
+    di->bwd_attr[aslot] = true;
   }
   const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
-  rb::bwd_kernel<<<grid, rb::NUM_THREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+  rb::bwd_kernel<HD><<<grid, rb::NUM_THREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
   if ((st = launch_status()) != RA_OK) return st;
 
   // 3. dQ = scale * accumulator -> bf16 (or added to dq32)
   if (dq32) {
-    const long long n4 = BH * S * rb::HD / 4;
+    const long long n4 = BH * S * HD / 4;
     const long long ablocks = (n4 + 255) / 256;
     if (ablocks > INT_MAX) return RA_ERR_SHAPE;
     rb::bwd_accum_dq_kernel<<<static_cast<int>(ablocks), 256, 0, stream>>>(dq_acc, dq32, n4, scale);
     return launch_status();
   }
-  const long long n8 = BH * S * rb::HD / 8;
+  const long long n8 = BH * S * HD / 8;
   const long long cblocks = (n8 + 255) / 256;
   if (cblocks > INT_MAX) return RA_ERR_SHAPE;
   rb::bwd_convert_kernel<<<static_cast<int>(cblocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8,
@@ -524,22 +526,30 @@ size_t ring_attn_bwd_workspace_size(int B, int H, int S, int Dh) {
   return bwd_workspace(static_cast<long long>(B) * H, S, Dh).total;
 }
 
-int ring_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                  void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D, int causal, void* workspace,
-                  size_t workspace_bytes, ra_stream stream) {
+int ring_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D, int causal, float scale,
+                     void* workspace, size_t workspace_bytes, ra_stream stream) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return RA_ERR_ARG;
   int st = check_shape(B, H, S, Dh, D);
   if (st != RA_OK) return st;
-  if (Dh != ra::bwd::HD) return RA_ERR_SHAPE;
+  if (Dh != 128 && Dh != 64) return RA_ERR_SHAPE;
   for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(dq), static_cast<const void*>(dk),
                           static_cast<const void*>(dv)})
     if (!aligned16(ptr)) return RA_ERR_ALIGN;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < ring_attn_bwd_workspace_size(B, H, S, Dh))
     return RA_ERR_WORKSPACE;
-  const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
-  return bwd_bf16(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, workspace,
-                  static_cast<cudaStream_t>(stream));
+  const float sc = (scale > 0.f && std::isfinite(scale)) ? scale : 1.0f / std::sqrt(static_cast<float>(Dh));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return Dh == 128 ? bwd_bf16<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, workspace, s)
+                   : bwd_bf16<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, workspace, s);
+}
+
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  void* dq, void* dk, void* dv, int B, int H, int S, int Dh, int D, int causal, void* workspace,
+                  size_t workspace_bytes, ra_stream stream) {
+  return ring_attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, Dh, D, causal, 0.f, workspace,
+                          workspace_bytes, stream);
 }
 
 int ring_attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -548,7 +558,7 @@ int ring_attn_bwd_accumulate(const void* q, const void* k, const void* v, const 
   if (!q || !k || !v || !o || !lse || !dO || !dq32 || !dk32 || !dv32) return RA_ERR_ARG;
   int st = check_shape(B, H, S, Dh, D);
   if (st != RA_OK) return st;
-  if (Dh != ra::bwd::HD) return RA_ERR_SHAPE;
+  if (Dh != 128 && Dh != 64) return RA_ERR_SHAPE;
   for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(dq32), static_cast<const void*>(dk32),
                           static_cast<const void*>(dv32)})
     if (!aligned16(ptr)) return RA_ERR_ALIGN;
@@ -556,8 +566,11 @@ int ring_attn_bwd_accumulate(const void* q, const void* k, const void* v, const 
       workspace_bytes < ring_attn_bwd_workspace_size(B, H, S, Dh))
     return RA_ERR_WORKSPACE;
   const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
-  return bwd_bf16(q, k, v, o, lse, dO, nullptr, nullptr, nullptr, B, H, S, D, causal, sc, workspace,
-                  static_cast<cudaStream_t>(stream), dq32, dk32, dv32);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return Dh == 128 ? bwd_bf16<128>(q, k, v, o, lse, dO, nullptr, nullptr, nullptr, B, H, S, D, causal, sc, workspace,
+                                   s, dq32, dk32, dv32)
+                   : bwd_bf16<64>(q, k, v, o, lse, dO, nullptr, nullptr, nullptr, B, H, S, D, causal, sc, workspace,
+                                  s, dq32, dk32, dv32);
 }
 
 int ring_attn_bwd_visit_tiles(int S, int D, int causal, int k0, int tile_rows, int* tiles, int max_tiles) {
@@ -618,7 +631,7 @@ int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return RA_ERR_ARG;
   int st = check_shape(B, H, S, Dh, D);
   if (st != RA_OK) return st;
-  if (Dh != ra::bwd::HD) return RA_ERR_SHAPE;
+  if (Dh != 128 && Dh != 64) return RA_ERR_SHAPE;
   for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(dq), static_cast<const void*>(dk),
                           static_cast<const void*>(dv)})
     if (!aligned16(ptr)) return RA_ERR_ALIGN;
@@ -628,8 +641,9 @@ int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch)) != RA_OK) return st;
   const float sc = 1.0f / std::sqrt(static_cast<float>(Dh));
-  return bwd_bf16(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, scratch,
-                  static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return Dh == 128 ? bwd_bf16<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, scratch, s)
+                   : bwd_bf16<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, scratch, s);
 }
 
 }  // extern "C"

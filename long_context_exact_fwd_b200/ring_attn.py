@@ -41,6 +41,8 @@ _split_ws = _sig("ring_attn_fwd_split_workspace_size", _sz, _i, _i, _i, _i, _i)
 _fwd_split = _sig("ring_attn_fwd_split", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
 _fwd_partial = _sig("ring_attn_fwd_partial", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _bwd = _sig("ring_attn_bwd", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp)
+_bwd_ex = _sig("ring_attn_bwd_ex", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp,
+               _sz, _vp)
 _merge_ex = _sig("ring_attn_merge_ex", _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp)
 _ring_order = _sig("ring_attn_ring_order", _i, _i, _i, _i, _ip, _i)
 _visit_tiles = _sig("ring_attn_visit_tiles", _i, _i, _i, _i, _i, _i, _ip, _i)
@@ -207,8 +209,9 @@ def bwd_workspace_bytes(B: int, H: int, S: int, Dh: int) -> int:
 
 
 def bwd(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=None,
-        workspace: Optional[torch.Tensor] = None, stream=None):
-    """Ring-attention backward (bf16).  Returns (dq, dk, dv), each [B, H, S, Dh] bf16."""
+        workspace: Optional[torch.Tensor] = None, stream=None, scale: Optional[float] = None):
+    """Ring-attention backward (bf16, Dh 64 or 128; ring_attn_bwd_ex).  `scale` must be the
+    forward's (None: 1/sqrt(Dh)).  Returns (dq, dk, dv), each [B, H, S, Dh] bf16."""
     B, H, S, Dh = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
         _need(t, name, torch.bfloat16, q.shape)
@@ -222,10 +225,11 @@ def bwd(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=None, dv=N
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     _need(workspace, "workspace")
-    code = _bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, Dh, D, 1 if causal else 0,
-                workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
-    _check(code, "ring_attn_bwd")
+    code = _bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                   dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, Dh, D, 1 if causal else 0,
+                   float(scale) if scale else 0.0, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                   _stream(stream))
+    _check(code, "ring_attn_bwd_ex")
     return dq, dk, dv
 
 

@@ -75,6 +75,25 @@ def test_merge_and_bwd_argument_errors(ra):
     assert ra.bwd_workspace_bytes(0, 2, 256, 128) == 0
 
 
+def test_backward_ex_argument_errors(ra):
+    f = ra.raw.ring_attn_bwd_ex
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    big = 1 << 30
+    args = lambda **kw: [P(kw.get("q", 256))] + [P(256)] * 8 + [1, 2, kw.get("S", 256), kw.get("Dh", 128),
+                                                                 kw.get("D", 4), 1, ctypes.c_float(0.3),
+                                                                 P(kw.get("ws", 256)),
+                                                                 ctypes.c_size_t(kw.get("wsb", big)), P(0)]
+    assert f(*args(q=0)) == ra.RA_ERR_ARG
+    assert f(*args(Dh=96)) == ra.RA_ERR_SHAPE          # backward kernels: Dh 64 and 128
+    assert f(*args(S=250)) == ra.RA_ERR_SHAPE          # uneven ring split
+    assert f(*args(q=264)) == ra.RA_ERR_ALIGN
+    assert f(*args(ws=0)) == ra.RA_ERR_WORKSPACE
+    assert f(*args(ws=272)) == ra.RA_ERR_WORKSPACE     # not 256-byte aligned
+    assert f(*args(wsb=16)) == ra.RA_ERR_WORKSPACE     # too small
+    assert ra.bwd_workspace_bytes(1, 2, 256, 64) >= 1 * 2 * 256 * 64 * 4
+
+
 def test_split_forward_workspace_and_argument_errors(ra):
     rows = 1 * 2 * 1000
     lse_block = (rows * 4 + 255) // 256 * 256
@@ -124,7 +143,7 @@ def test_accumulating_backward_argument_errors(ra):
     assert f(*args(q=0)) == ra.RA_ERR_ARG
     assert f(*args(dq32=0)) == ra.RA_ERR_ARG
     assert f(*args(S=1001)) == ra.RA_ERR_SHAPE
-    assert f(*args(Dh=64)) == ra.RA_ERR_SHAPE          # the backward is Dh = 128 only
+    assert f(*args(Dh=96)) == ra.RA_ERR_SHAPE          # backward kernels: Dh 64 and 128
     assert f(*args(dq32=264)) == ra.RA_ERR_ALIGN
     assert f(*args(ws=0)) == ra.RA_ERR_WORKSPACE
     assert f(*args(ws=272)) == ra.RA_ERR_WORKSPACE

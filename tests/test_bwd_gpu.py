@@ -19,10 +19,10 @@ def ra():
     return ring_attn
 
 
-def _fwd_bwd(ra, inp, D, causal):
+def _fwd_bwd(ra, inp, D, causal, scale=None):
     q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
-    o, lse = ra.fwd(q, k, v, D, causal)
-    dq, dk, dv = ra.bwd(q, k, v, o, lse, do, D, causal)
+    o, lse = ra.fwd(q, k, v, D, causal, scale=scale)
+    dq, dk, dv = ra.bwd(q, k, v, o, lse, do, D, causal, scale=scale)
     assert ra.device_status() == 0
     return [t.float().cpu().numpy() for t in (dq, dk, dv)]
 
@@ -89,3 +89,41 @@ def test_bwd_workspace_errors(ra):
     with pytest.raises(ra.RingAttnError) as e:
         ra.bwd(q, k, v, o, lse, do, 2, True, workspace=small)
     assert e.value.code == ra.RA_ERR_WORKSPACE
+
+
+# Dh = 64: ragged S (not a multiple of the 128-row tiles), D = 3..8 ring blocks
+BWD_SHAPES_64 = [(1, 2, 300, 64, 3), (2, 1, 129, 64, 3), (1, 1, 1000, 64, 8), (1, 3, 640, 64, 5),
+                 (1, 2, 2048, 64, 4), (1, 1, 777, 64, 7)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H,S,Dh,D", BWD_SHAPES_64)
+def test_bwd_head_dim_64(ra, B, H, S, Dh, D, causal):
+    inp = random_qkv(B, H, S, Dh, seed=2000 + S + D, with_do=True)
+    got = _fwd_bwd(ra, inp, D, causal)
+    ref = oracle.attn_bwd_heads(inp["q"], inp["k"], inp["v"], inp["do"], causal)
+    _check(got, ref)
+
+
+@pytest.mark.parametrize("Dh", [64, 128])
+@pytest.mark.parametrize("scale", [0.05, 0.2])
+def test_bwd_with_caller_scale(ra, Dh, scale):
+    """ring_attn_bwd_ex with the scale the forward used, against the oracle's gradient at that
+    scale (a wrong or ignored scale moves P, dQ and dK well past the bar)."""
+    inp = random_qkv(1, 2, 700, Dh, seed=3000 + Dh, with_do=True)
+    got = _fwd_bwd(ra, inp, 4, True, scale=scale)
+    ref = oracle.attn_bwd_heads(inp["q"], inp["k"], inp["v"], inp["do"], True, scale=scale)
+    _check(got, ref)
+
+
+def test_bwd_accumulate_head_dim_64(ra):
+    """ring_attn_bwd_accumulate at Dh = 64: two calls add twice the gradient in float32."""
+    inp = random_qkv(1, 2, 500, 64, seed=17, with_do=True)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = ra.fwd(q, k, v, 5, True)
+    acc = [torch.zeros(q.shape, dtype=torch.float32, device="cuda") for _ in range(3)]
+    for _ in range(2):
+        ra.bwd_accumulate(q, k, v, o, lse, do, 5, True, *acc)
+    assert ra.device_status() == 0
+    ref = oracle.attn_bwd_heads(inp["q"], inp["k"], inp["v"], inp["do"], True)
+    _check([(a / 2).cpu().numpy() for a in acc], ref)
