@@ -23,9 +23,13 @@ algorithm against the plain definition; the key-subset attention against a brute
 loop and, over a key partition, merged to the full result; the block-pair gradient with
 full-row statistics summed over block pairs to the full gradient; the per-head wrappers
 (forward and backward) against per-slice calls and, for the backward over several batch
-entries and heads, against batched torch float64 autograd.  No function here is
-"parity unpinned".
+entries and heads, against batched torch float64 autograd.  The blockwise feedforward
+(``ffn.py``): GELU against the normal CDF's tabulated values and its odd-part identity, the
+two-matrix feedforward against a scalar loop and torch float64 library calls, the head-to-token
+layout against an explicit index loop, and blockwise = whole sequence for every block size.
+No function here is "parity unpinned".
 """
+from .ffn import ffn_blockwise, ffn_rows, gelu, heads_to_tokens  # noqa: F401
 from .attention import (  # noqa: F401
     attn_fwd,
     attn_fwd_keys,
