@@ -14,7 +14,9 @@ the max over ranks.
 
 On one GPU the default run then times the forward alone on the S=32K (score outliers) and
 S=128K workloads, inputs resident, each over at least half a second with its own clock record,
-and reports them under kernels["ring_attn_fwd@<workload>"] (--no-gate skips them).
+and reports them under kernels["ring_attn_fwd@<workload>"]; then the blockwise feedforward that
+follows attention (ring_attn_ffn_fwd, h = 2048, f = 8192, D = 8 blocks of 2048 tokens) under
+kernels["ring_attn_ffn@s16k"] (--no-gate skips all three).
 
 End to end ("e2e"): the same steps through the public API with pinned host inputs copied in and
 the step's results (dQ, dK, dV; or O, LSE) copied out every step.  "value" overlaps step i + 1's
@@ -99,6 +101,7 @@ def _peaks():
 KERNEL_SOURCES = {
     "fwd_kernel": ("fwd_sm100.cuh", "ra_sm100.cuh", "ra_schedule.h", "ra_work.cuh", "ring_attn.cu"),
     "bwd_kernel": ("bwd_sm100.cuh", "ra_sm100.cuh", "ra_schedule.h", "ra_work.cuh", "ring_attn.cu"),
+    "gemm_kernel": ("ffn_sm100.cuh", "ra_sm100.cuh", "ring_attn.cu"),
 }
 
 
@@ -318,6 +321,60 @@ def time_fwd_leg(w: Workload, dev, stream, warmup: int):
             "clocks": clocks.summary()}
 
 
+def time_ffn_leg(w: Workload, dev, stream, warmup: int):
+    """The blockwise feedforward after attention on one GPU (ring_attn_ffn_fwd: every ring block
+    in turn, one block's hidden activation alive): x = the workload's attention output layout
+    [B, H, S, Dh] (seeded N(0,1) bf16 standing in for it), h = H * Dh, f = 4h, seeded weights.
+    FLOPs 4 * B * S * h * f (two matrices); timed per call over at least MIN_TIMED_S."""
+    import torch
+    from long_context_exact_fwd_b200 import ring_attn as ra
+    from long_context_exact_fwd_b200.workloads import ffn_weights
+    x = make_inputs(w)["q"].to(dev)
+    h = w.H * w.Dh
+    f = 4 * h
+    wt = {n: t.to(dev) for n, t in ffn_weights(h, f, seed=w.seed + 77).items()}
+    y = torch.empty((w.B, w.S, h), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(ra.ffn_workspace_bytes(w.B, w.S, w.D, f), dtype=torch.uint8, device=dev)
+
+    def run():
+        ra.ffn(x, wt["w1"], wt["b1"], wt["w2"], wt["b2"], w.D, out=y, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    n = max(3, math.ceil(MIN_TIMED_S * 1e3 / e0.elapsed_time(e1)))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(uuid) as clocks:
+        t_wall = time.perf_counter()
+        for a, b in evs:
+            a.record(stream)
+            run()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall
+    if ra.device_status(stream) != 0:
+        raise RuntimeError("device status not clean after the feedforward")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    peaks, src = _peaks()
+    sustained = t_wall > 2.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    flops = 4.0 * w.B * w.S * h * f
+    del x, y, ws, wt
+    torch.cuda.empty_cache()
+    return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "frac": flops / (ms * 1e-3) / 1e12 / peak,
+            "peak": peak, "peak_source": f"{src} {'sustained' if sustained else 'burst'} bf16 dense",
+            "launches_timed": n, "timed_s": t_wall, "traffic": _traffic("gemm_kernel", "s16k_ffn"),
+            "config": {"B": w.B, "S": w.S, "h": h, "f": f, "D": w.D, "c": w.c, "flops": flops,
+                       "activation_bytes": 2 * w.B * w.c * f, "weights": f"seeded, seed {w.seed + 77}"},
+            "clocks": clocks.summary()}
+
+
 def run_ours(args, w: Workload):
     import torch
     import torch.distributed as dist
@@ -510,6 +567,7 @@ def run_ours(args, w: Workload):
         torch.cuda.empty_cache()
         for name in GATE_WORKLOADS:
             gate[name] = time_fwd_leg(WORKLOADS[name], dev, stream, args.warmup)
+        ffn_leg = time_ffn_leg(w, dev, stream, args.warmup)
 
     if rank == 0:
         peaks, src = _peaks()
@@ -523,6 +581,8 @@ def run_ours(args, w: Workload):
                                         "frac": w.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak}
         for name, leg in gate.items():
             kernels[f"ring_attn_fwd@{name}"] = leg
+        if gate:
+            kernels["ring_attn_ffn@s16k"] = ffn_leg
         dom = "ring_attn_bwd" if (w.backward and b_ms >= f_ms) else "ring_attn_fwd"
         dom_kernel = "bwd_kernel" if dom == "ring_attn_bwd" else "fwd_kernel"
         achieved = kernels[dom]["tflops"]

@@ -228,6 +228,51 @@ RA_API int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, co
 RA_API size_t ring_attn_bwd_noalloc_max_bytes(void);
 
 /*
+ * ring_attn_ffn_workspace_size -- bytes of device workspace the blockwise feedforward needs: one
+ * ring block's hidden activation, bf16 [B][S / D][f], rounded up to 256 bytes.  Returns 0 for
+ * invalid sizes.
+ */
+RA_API size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f);
+
+/*
+ * ring_attn_ffn_block -- the feedforward that follows attention, for ring block r only
+ * (page "精读笔记 ...", §2.2: blockwise parallel transformers compute the feedforward of each
+ * attention sub-layer block by block, so the largest activation is one block's hidden layer
+ * -- 2bsh instead of 8bsh bytes; §3.5 Algorithm 1: per layer, each host's block goes through
+ * attention and then the feedforward).  With x the block's attention output, heads side by side
+ * per token (x[b, s, head * Dh + d] = o[b, head, s, d], h = H * Dh):
+ *   y = gelu(x W1^T + b1) W2^T + b2,   gelu(u) = u * Phi(u) (exact form; the pages name no
+ *   activation, and 8bsh bytes of bf16 activation is a hidden layer of f = 4h, the default).
+ *   o         [B][H][S][Dh] bf16 attention output (ring_attn_fwd's o), read in place.
+ *   B, H, S, Dh, D  as ring_attn_fwd (Dh 64 or 128); the block is tokens [r c, r c + c), c = S/D.
+ *   r         ring block, 0 <= r < D (else RA_ERR_ARG).
+ *   w1        [f][h] bf16 (the first layer's weight in [out][in] layout), b1 [f] float32.
+ *   w2        [h][f] bf16, b2 [h] float32.
+ *   f         hidden width, a positive multiple of 64.
+ *   y         [B][S][h] bf16; only the block's rows are written.
+ *   workspace >= ring_attn_ffn_workspace_size(B, S, D, f) bytes of device memory, 256-byte
+ *             aligned: the block's hidden activation gelu(x W1^T + b1), rounded to bf16 (the
+ *             activation the pages' memory count stores), overwritten by every call.
+ * Two launches on `stream` (tcgen05 GEMM with a bias + GELU epilogue, then with a bias
+ * epilogue); float32 accumulation.  Pointers 16-byte aligned.  Errors: RA_ERR_ARG (null
+ * pointer, f <= 0, r out of range), RA_ERR_SHAPE (S % D, Dh, f % 64, sizes), RA_ERR_ALIGN,
+ * RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ */
+RA_API int ring_attn_ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r, const void* w1,
+                               const float* b1, const void* w2, const float* b2, int f, void* y, void* workspace,
+                               size_t workspace_bytes, ra_stream stream);
+
+/*
+ * ring_attn_ffn_fwd -- ring_attn_ffn_block for every ring block r = 0 .. D-1 in turn on
+ * `stream`, reusing the one block-sized workspace: the whole sequence's feedforward with one
+ * block's hidden activation alive at a time.  Arguments and errors as ring_attn_ffn_block
+ * (without r).
+ */
+RA_API int ring_attn_ffn_fwd(const void* o, int B, int H, int S, int Dh, int D, const void* w1, const float* b1,
+                             const void* w2, const float* b2, int f, void* y, void* workspace, size_t workspace_bytes,
+                             ra_stream stream);
+
+/*
  * ring_attn_merge -- combine P normalised partial outputs through their log-sum-exp
  * (page "精读笔记 ...", §3.1: blocks may be combined in any order when their statistics are
  * combined with rescaling; page "RingAttention large-context attention", 架构与算法: the

@@ -16,6 +16,7 @@
 #include "fwd_f32.cuh"
 #include "merge.cuh"
 #include "bwd_sm100.cuh"
+#include "ffn_sm100.cuh"
 
 namespace {
 
@@ -60,6 +61,7 @@ struct DevInfo {
   // written by any host thread, hence atomic (setting an attribute twice is harmless)
   std::atomic<bool> fwd_attr[4] = {false, false, false, false};
   std::atomic<bool> bwd_attr[2] = {false, false};   // [HD 128, HD 64]
+  std::atomic<bool> ffn_attr{false};
 };
 
 std::mutex g_dev_mu;
@@ -126,12 +128,18 @@ int check_shape(int B, int H, int S, int Dh, int D) {
   return RA_OK;
 }
 
-// Heads whose per-head streamed operands (`bytes_per_head`) fit together in ~48 MiB of L2.
+// Heads whose per-head streamed operands (`bytes_per_head`) fit together in `mib` MiB of L2.
 #ifndef RA_L2_GROUP_MIB
-#define RA_L2_GROUP_MIB 48
+#define RA_L2_GROUP_MIB 48          // backward: Q + dO of the heads in flight
 #endif
-int heads_per_l2_group(long long BH, long long bytes_per_head) {
-  const long long g = (static_cast<long long>(RA_L2_GROUP_MIB) << 20) / (bytes_per_head > 0 ? bytes_per_head : 1);
+#ifndef RA_FWD_L2_GROUP_MIB
+#define RA_FWD_L2_GROUP_MIB 48      // forward: K + V of the heads in flight (0: all heads) ...
+#endif
+#ifndef RA_FWD_L2_GROUP_ABOVE_MIB
+#define RA_FWD_L2_GROUP_ABOVE_MIB 256   // ... once K + V of all heads exceed this (about 2x L2)
+#endif
+int heads_per_l2_group(long long BH, long long bytes_per_head, long long mib = RA_L2_GROUP_MIB) {
+  const long long g = (mib << 20) / (bytes_per_head > 0 ? bytes_per_head : 1);
   return static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
 }
 
@@ -166,9 +174,15 @@ int fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, i
   const long long items = BH * p.n_pairs * n_parts;
   if (items > INT_MAX) return RA_ERR_SHAPE;
   p.n_items = static_cast<int>(items);
-  // All heads interleaved: with dynamic scheduling this measured best per cycle at S = 16K
-  // and 32K; grouping heads for L2 reuse pays off in the backward only.
-  p.hgroup = static_cast<int>(BH);
+  // Heads grouped so the K and V of the heads in flight fit in ~48 MiB of L2, once all heads'
+  // K and V are well beyond L2.  Measured on B200 (0.5 s regions, clocks under the power cap):
+  // S = 32K, 32 heads 1012 -> 1054 TFLOP/s and S = 128K, 8 heads 1083 -> 1095 (the DRAM traffic
+  // falls and the SM clock rises ~100 MHz); at S = 16K, 16 heads (128 MiB of K and V) all heads
+  // interleaved stays best (1012 against 962).
+  const long long kv_head = 4ll * S * HD;   // K + V bytes of one head
+  p.hgroup = (RA_FWD_L2_GROUP_MIB > 0 && BH * kv_head > (static_cast<long long>(RA_FWD_L2_GROUP_ABOVE_MIB) << 20))
+                 ? heads_per_l2_group(BH, kv_head, RA_FWD_L2_GROUP_MIB)
+                 : static_cast<int>(BH);
   p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -644,6 +658,129 @@ int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return Dh == 128 ? bwd_bf16<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, scratch, s)
                    : bwd_bf16<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, S, D, causal, sc, scratch, s);
+}
+
+}  // extern "C"
+
+// --- blockwise feedforward after attention ------------------------------------------------
+namespace {
+
+size_t ffn_workspace(int B, int S, int D, int f) {
+  return align256(static_cast<size_t>(B) * (S / D) * f * 2);
+}
+
+// Arguments shared by the two feedforward entry points; RA_OK when usable.
+int ffn_check(const void* o, int B, int H, int S, int Dh, int D, const void* w1, const float* b1, const void* w2,
+              const float* b2, int f, void* y, void* workspace, size_t workspace_bytes) {
+  if (!o || !w1 || !b1 || !w2 || !b2 || !y) return RA_ERR_ARG;
+  if (f <= 0) return RA_ERR_ARG;
+  int st = check_shape(B, H, S, Dh, D);
+  if (st != RA_OK) return st;
+  if (Dh != 64 && Dh != 128) return RA_ERR_SHAPE;
+  if (f % 64 != 0) return RA_ERR_SHAPE;
+  const long long h = static_cast<long long>(H) * Dh;
+  if (h > (1 << 20) || f > (1 << 24)) return RA_ERR_SHAPE;
+  if (static_cast<double>(B) * S * (h > f ? h : f) > 9.0e18 / 4) return RA_ERR_SHAPE;
+  for (const void* ptr : {o, w1, w2, static_cast<const void*>(b1), static_cast<const void*>(b2),
+                          static_cast<const void*>(y)})
+    if (!aligned16(ptr)) return RA_ERR_ALIGN;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < ffn_workspace(B, S, D, f))
+    return RA_ERR_WORKSPACE;
+  return RA_OK;
+}
+
+int ffn_gemm(DevInfo* di, const CUtensorMap& ma, const CUtensorMap& mb, ra::ffn::Params& p, cudaStream_t stream) {
+  namespace rf = ra::ffn;
+  p.m_tiles_per_b = (p.rows + rf::BM - 1) / rf::BM;
+  p.n_tiles = (p.N + rf::BN - 1) / rf::BN;
+  const long long items = static_cast<long long>(p.m_tiles) * p.n_tiles;
+  if (items > INT_MAX) return RA_ERR_SHAPE;
+  p.n_items = static_cast<int>(items);
+  constexpr int smem = rf::Layout::ALLOC;
+  if (!di->ffn_attr) {
+    const cudaError_t e = cudaFuncSetAttribute(rf::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(ffn smem)");
+    di->ffn_attr = true;
+  }
+  const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
+  rf::gemm_kernel<<<grid, rf::NUM_THREADS, smem, stream>>>(ma, mb, p);
+  return launch_status();
+}
+
+// Feedforward of ring block r: GEMM 1 (attention output -> hidden activation Z in the
+// workspace, bias + GELU) then GEMM 2 (Z -> y rows of the block, bias).
+int ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r, const void* w1, const float* b1,
+              const void* w2, const float* b2, int f, void* y, void* workspace, cudaStream_t stream) {
+  int st = RA_OK;
+  DevInfo* di = dev_info(&st);
+  if (!di) return st;
+  const int c = S / D;
+  const int h = H * Dh;
+  ra::ffn::Params p1{};
+  p1.K = h;
+  p1.N = f;
+  p1.rows = c;
+  p1.m_tiles = B * ((c + ra::ffn::BM - 1) / ra::ffn::BM);
+  p1.a_kdim = Dh;
+  p1.a_row0 = r * c;
+  p1.a_outer_per_b = H;
+  p1.c_rows_per_b = c;
+  p1.c_row0 = 0;
+  p1.ldc = f;
+  p1.bias = b1;
+  p1.c = static_cast<__nv_bfloat16*>(workspace);
+  p1.gelu = 1;
+  CUtensorMap ma, mb;
+  if ((st = make_map(&ma, o, static_cast<long long>(B) * H, S, Dh, ra::ffn::BM)) != RA_OK) return st;
+  if ((st = make_map(&mb, w1, 1, f, h, ra::ffn::BN)) != RA_OK) return st;
+  if ((st = ffn_gemm(di, ma, mb, p1, stream)) != RA_OK) return st;
+
+  ra::ffn::Params p2 = p1;
+  p2.K = f;
+  p2.N = h;
+  p2.a_kdim = f;
+  p2.a_row0 = 0;
+  p2.a_outer_per_b = 1;
+  p2.c_rows_per_b = S;
+  p2.c_row0 = static_cast<long long>(r) * c;
+  p2.ldc = h;
+  p2.bias = b2;
+  p2.c = static_cast<__nv_bfloat16*>(y);
+  p2.gelu = 0;
+  if ((st = make_map(&ma, workspace, B, c, f, ra::ffn::BM)) != RA_OK) return st;
+  if ((st = make_map(&mb, w2, 1, h, f, ra::ffn::BN)) != RA_OK) return st;
+  return ffn_gemm(di, ma, mb, p2, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f) {
+  if (B <= 0 || S <= 0 || D <= 0 || D > S || S % D != 0 || f <= 0) return 0;
+  return ffn_workspace(B, S, D, f);
+}
+
+int ring_attn_ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r, const void* w1, const float* b1,
+                        const void* w2, const float* b2, int f, void* y, void* workspace, size_t workspace_bytes,
+                        ra_stream stream) {
+  int st = ffn_check(o, B, H, S, Dh, D, w1, b1, w2, b2, f, y, workspace, workspace_bytes);
+  if (st != RA_OK) return st;
+  if (r < 0 || r >= D) return RA_ERR_ARG;
+  return ffn_block(o, B, H, S, Dh, D, r, w1, b1, w2, b2, f, y, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_ffn_fwd(const void* o, int B, int H, int S, int Dh, int D, const void* w1, const float* b1,
+                      const void* w2, const float* b2, int f, void* y, void* workspace, size_t workspace_bytes,
+                      ra_stream stream) {
+  int st = ffn_check(o, B, H, S, Dh, D, w1, b1, w2, b2, f, y, workspace, workspace_bytes);
+  if (st != RA_OK) return st;
+  for (int r = 0; r < D; ++r) {
+    st = ffn_block(o, B, H, S, Dh, D, r, w1, b1, w2, b2, f, y, workspace, static_cast<cudaStream_t>(stream));
+    if (st != RA_OK) return st;
+  }
+  return RA_OK;
 }
 
 }  // extern "C"

@@ -56,6 +56,9 @@ _bwd_acc = _sig("ring_attn_bwd_accumulate", _i, _vp, _vp, _vp, _vp, _vp, _vp, _v
                 _i, _vp, _sz, _vp)
 _bwd_noalloc = _sig("ring_attn_bwd_noalloc", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
 _noalloc_max = _sig("ring_attn_bwd_noalloc_max_bytes", _sz)
+_ffn_ws = _sig("ring_attn_ffn_workspace_size", _sz, _i, _i, _i, _i)
+_ffn_fwd = _sig("ring_attn_ffn_fwd", _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _sz, _vp)
+_ffn_block = _sig("ring_attn_ffn_block", _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _sz, _vp)
 _exp2_check = _sig("ring_attn_exp2_check", _i, _vp, _vp, _vp, ctypes.c_longlong, _vp)
 _wait_selftest = _sig("ring_attn_wait_selftest", _i, ctypes.c_longlong, _vp)
 
@@ -273,6 +276,43 @@ def bwd_noalloc(q, k, v, o, lse, do, D: int, causal: bool = True, dq=None, dk=No
                         _stream(stream))
     _check(code, "ring_attn_bwd_noalloc")
     return dq, dk, dv
+
+
+def ffn_workspace_bytes(B: int, S: int, D: int, f: int) -> int:
+    return int(_ffn_ws(B, S, D, f))
+
+
+def ffn(o: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: torch.Tensor, D: int,
+        block: Optional[int] = None, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+        stream=None) -> torch.Tensor:
+    """Blockwise feedforward after attention (ring_attn_ffn_fwd, or ring_attn_ffn_block for one
+    ring block): o [B, H, S, Dh] bf16 attention output; w1 [f, H*Dh], w2 [H*Dh, f] bf16; b1 [f],
+    b2 [H*Dh] float32.  Returns y [B, S, H*Dh] bf16 = gelu(x w1^T + b1) w2^T + b2 with
+    x[b, s] the heads of token s side by side (only block `block`'s rows are written when given)."""
+    if o.dim() != 4:
+        raise ValueError("o must be [B, H, S, Dh]")
+    B, H, S, Dh = o.shape
+    h, f = H * Dh, w1.shape[0]
+    _need(o, "o", torch.bfloat16)
+    _need(w1, "w1", torch.bfloat16, (f, h))
+    _need(w2, "w2", torch.bfloat16, (h, f))
+    _need(b1, "b1", torch.float32, (f,))
+    _need(b2, "b2", torch.float32, (h,))
+    out = torch.empty((B, S, h), dtype=torch.bfloat16, device=o.device) if out is None else out
+    _need(out, "out", torch.bfloat16, (B, S, h))
+    if workspace is None:
+        workspace = torch.empty(max(ffn_workspace_bytes(B, S, D, f), 1), dtype=torch.uint8, device=o.device)
+    _need(workspace, "workspace")
+    wsb = workspace.numel() * workspace.element_size()
+    if block is None:
+        code = _ffn_fwd(o.data_ptr(), B, H, S, Dh, D, w1.data_ptr(), b1.data_ptr(), w2.data_ptr(), b2.data_ptr(), f,
+                        out.data_ptr(), workspace.data_ptr(), wsb, _stream(stream))
+        _check(code, "ring_attn_ffn_fwd")
+    else:
+        code = _ffn_block(o.data_ptr(), B, H, S, Dh, D, int(block), w1.data_ptr(), b1.data_ptr(), w2.data_ptr(),
+                          b2.data_ptr(), f, out.data_ptr(), workspace.data_ptr(), wsb, _stream(stream))
+        _check(code, "ring_attn_ffn_block")
+    return out
 
 
 def bwd_noalloc_max_bytes() -> int:

@@ -148,6 +148,21 @@ def sample_rows(w: Workload, n: Optional[int] = None) -> torch.Tensor:
     return rows
 
 
+def ffn_weights(h: int, f: int, seed: int, dtype=torch.bfloat16, device: str = "cpu") -> Dict[str, torch.Tensor]:
+    """Seeded synthetic feedforward weights (no trained model exists here): a CPU generator
+    seeded ``seed`` draws, in float32 and in this order, W1 [f, h] ~ N(0, 1/h), b1 [f] ~
+    N(0, 0.1^2), W2 [h, f] ~ N(0, 1/f), b2 [h] ~ N(0, 0.1^2) (fan-in scaling keeps the
+    activations O(1)); the weights are cast to ``dtype``, the biases stay float32."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    w1 = torch.randn((f, h), generator=g, dtype=torch.float32) * h ** -0.5
+    b1 = torch.randn((f,), generator=g, dtype=torch.float32) * 0.1
+    w2 = torch.randn((h, f), generator=g, dtype=torch.float32) * f ** -0.5
+    b2 = torch.randn((h,), generator=g, dtype=torch.float32) * 0.1
+    return {"w1": w1.to(dtype).contiguous().to(device), "b1": b1.to(device),
+            "w2": w2.to(dtype).contiguous().to(device), "b2": b2.to(device)}
+
+
 def random_qkv(B: int, H: int, S: int, Dh: int, seed: int, dtype=torch.bfloat16,
                with_do: bool = False, device: str = "cpu") -> Dict[str, torch.Tensor]:
     """Ad-hoc seeded N(0,1) tensors for shape sweeps (same recipe, no outliers)."""

@@ -94,6 +94,30 @@ def test_backward_ex_argument_errors(ra):
     assert ra.bwd_workspace_bytes(1, 2, 256, 64) >= 1 * 2 * 256 * 64 * 4
 
 
+def test_ffn_argument_errors(ra):
+    f = ra.raw.ring_attn_ffn_block
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    big = 1 << 40
+    args = lambda **kw: [P(kw.get("o", 256)), 1, 2, kw.get("S", 300), kw.get("Dh", 64), kw.get("D", 3),
+                         kw.get("r", 0), P(256), P(kw.get("b1", 256)), P(256), P(256), kw.get("f", 256), P(256),
+                         P(kw.get("ws", 256)), ctypes.c_size_t(kw.get("wsb", big)), P(0)]
+    assert f(*args(o=0)) == ra.RA_ERR_ARG
+    assert f(*args(r=3)) == ra.RA_ERR_ARG           # ring block out of range
+    assert f(*args(r=-1)) == ra.RA_ERR_ARG
+    assert f(*args(f=0)) == ra.RA_ERR_ARG
+    assert f(*args(f=100)) == ra.RA_ERR_SHAPE       # hidden width: a multiple of 64
+    assert f(*args(Dh=96)) == ra.RA_ERR_SHAPE
+    assert f(*args(S=301)) == ra.RA_ERR_SHAPE       # uneven ring split
+    assert f(*args(b1=260)) == ra.RA_ERR_ALIGN
+    assert f(*args(ws=0)) == ra.RA_ERR_WORKSPACE
+    assert f(*args(wsb=100 * 256 * 2 - 1)) == ra.RA_ERR_WORKSPACE
+    # one block's hidden activation, bf16 [B][S/D][f], rounded up to 256 bytes
+    assert ra.ffn_workspace_bytes(1, 300, 3, 256) == 100 * 256 * 2
+    assert ra.ffn_workspace_bytes(2, 300, 3, 64) == (2 * 100 * 64 * 2 + 255) // 256 * 256
+    assert ra.ffn_workspace_bytes(1, 300, 7, 256) == 0
+
+
 def test_split_forward_workspace_and_argument_errors(ra):
     rows = 1 * 2 * 1000
     lse_block = (rows * 4 + 255) // 256 * 256
