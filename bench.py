@@ -633,6 +633,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gate", action="store_true",
                     help="skip the forward-only S=32K and S=128K legs timed after the default workload")
+    ap.add_argument("--ffn-only", action="store_true",
+                    help="time only the blockwise feedforward of the default workload's shape (one GPU) and "
+                         "print its record")
     ap.add_argument("--passes", type=int, default=0,
                     help="passes of the hot path per reported step (0: enough for a %.1f s timed region)"
                          % MIN_TIMED_S)
@@ -643,6 +646,12 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.ffn_only:
+        import torch
+        torch.cuda.set_device(0)
+        dev = torch.device("cuda", 0)
+        print(json.dumps({"ffn": time_ffn_leg(w, dev, torch.cuda.current_stream(dev), args.warmup)}), flush=True)
+        return 0
     return run_ours(args, w)
 
 
