@@ -228,9 +228,11 @@ RA_API int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, co
 RA_API size_t ring_attn_bwd_noalloc_max_bytes(void);
 
 /*
- * ring_attn_ffn_workspace_size -- bytes of device workspace the blockwise feedforward needs: one
- * ring block's hidden activation, bf16 [B][S / D][f], rounded up to 256 bytes.  Returns 0 for
- * invalid sizes.
+ * ring_attn_ffn_workspace_size -- bytes of device workspace the blockwise feedforward needs: two
+ * ring blocks' hidden activations, bf16 [2][B][S / D][f] (block r + 1's first product runs while
+ * block r's second drains), then 4 * B * ceil((S / D) / 128) 32-bit dependency counters, each
+ * region rounded up to 256 bytes.  Independent of D for a given block size: the activation alive
+ * is two blocks', never the sequence's.  Returns 0 for invalid sizes.
  */
 RA_API size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f);
 
@@ -251,22 +253,27 @@ RA_API size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f);
  *   f         hidden width, a positive multiple of 64.
  *   y         [B][S][h] bf16; only the block's rows are written.
  *   workspace >= ring_attn_ffn_workspace_size(B, S, D, f) bytes of device memory, 256-byte
- *             aligned: the block's hidden activation gelu(x W1^T + b1), rounded to bf16 (the
- *             activation the pages' memory count stores), overwritten by every call.
- * Two launches on `stream` (tcgen05 GEMM with a bias + GELU epilogue, then with a bias
- * epilogue); float32 accumulation.  Pointers 16-byte aligned.  Errors: RA_ERR_ARG (null
- * pointer, f <= 0, r out of range), RA_ERR_SHAPE (S % D, Dh, f % 64, sizes), RA_ERR_ALIGN,
- * RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ *             aligned: the hidden activation gelu(x W1^T + b1), rounded to bf16 (the activation
+ *             the pages' memory count stores), and the dependency counters; overwritten by every
+ *             call.
+ * A memset of the counters and one persistent launch on `stream`: tcgen05 tiles of both
+ * products (bias + GELU epilogue, then bias epilogue), float32 accumulation; a tile of the
+ * second product starts once the first product's tiles of its rows are stored.  Pointers
+ * 16-byte aligned.  Calls that overlap on the GPU must not share a workspace.  Errors:
+ * RA_ERR_ARG (null pointer, f <= 0, r out of range), RA_ERR_SHAPE (S % D, Dh, f % 64, sizes),
+ * RA_ERR_ALIGN, RA_ERR_WORKSPACE, RA_ERR_CUDA; RA_ERR_TIMEOUT in the device status word if a
+ * bounded wait gave up.
  */
 RA_API int ring_attn_ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r, const void* w1,
                                const float* b1, const void* w2, const float* b2, int f, void* y, void* workspace,
                                size_t workspace_bytes, ra_stream stream);
 
 /*
- * ring_attn_ffn_fwd -- ring_attn_ffn_block for every ring block r = 0 .. D-1 in turn on
- * `stream`, reusing the one block-sized workspace: the whole sequence's feedforward with one
- * block's hidden activation alive at a time.  Arguments and errors as ring_attn_ffn_block
- * (without r).
+ * ring_attn_ffn_fwd -- the feedforward of every ring block r = 0 .. D-1, in that order, in one
+ * persistent launch: block r + 1's first product overlaps block r's second, and the two
+ * block-sized activation buffers of the workspace alternate, so at most two blocks' hidden
+ * activations are alive, whatever the sequence length.  Arguments and errors as
+ * ring_attn_ffn_block (without r).
  */
 RA_API int ring_attn_ffn_fwd(const void* o, int B, int H, int S, int Dh, int D, const void* w1, const float* b1,
                              const void* w2, const float* b2, int f, void* y, void* workspace, size_t workspace_bytes,

@@ -1,29 +1,36 @@
-// Blockwise feedforward after attention, for sm_100a: a persistent TMA + tcgen05 GEMM with a
-// fused bias / GELU epilogue, run on one ring block of c tokens at a time.
+// Blockwise feedforward after attention, for sm_100a: one persistent TMA + tcgen05 launch that
+// runs both matrix products of every ring block, with the bias / GELU epilogue fused.
 //
 // Page "精读笔记 · Ring Attention with Blockwise Transformers for Near-Infinite Context", §2.2
 // (BPT): the feedforward of each attention sub-layer is computed block by block, so its largest
-// activation is one block's hidden layer instead of the whole sequence's (2bsh instead of 8bsh
+// activation is a block's hidden layer instead of the whole sequence's (2bsh instead of 8bsh
 // bytes); §3.5 Algorithm 1: per layer each host's block goes through attention, then the
 // feedforward.  Y = gelu(X W1^T + b1) W2^T + b2 with X the block's attention output, heads side
 // by side per token; GELU in its exact form x Phi(x) (the pages name no activation).
 //
-// One kernel computes C[m, n] = epi(sum_k A[m, k] B[n, k] + bias[n]) for one block:
-//   GEMM 1: A = the attention output O [B][H][S][Dh] read in place (token rows of the block,
-//           K index = head * Dh + d), B = W1 [f][h], epi = GELU, C = Z [B][c][f] (workspace);
-//   GEMM 2: A = Z, B = W2 [h][f], epi = identity, C = Y [B][S][h] rows of the block.
-// Both operands are K-major and arrive by 3-D TMA tile loads (128-byte swizzle, no multicast);
-// an A tile never crosses a batch entry, and rows past the block are loaded but not stored.
+// Work items (tiles of 128 rows x 256 columns), in this order, block after block:
+//   GEMM 1 of block r: A = the attention output O [B][H][S][Dh] read in place (token rows of the
+//           block; K index = head * Dh + d), B = W1 [f][h], epi = bias + GELU, C = Z_u [B][c][f];
+//   GEMM 2 of block r: A = Z_u, B = W2 [h][f], epi = bias, C = the block's rows of Y [B][S][h].
+// Z_u (u = block index in the launch mod 2) are two block-sized hidden activations in the
+// caller's workspace, so block r + 1's GEMM 1 runs while block r's GEMM 2 drains.  Dependencies,
+// through per-row-tile counters in the workspace (cleared before the launch):
+//   ready[u][m]    GEMM 1 tiles of row tile m that have stored their Z columns; a GEMM 2 tile of
+//                  row tile m starts loading Z once all column tiles of its block are in;
+//   consumed[u][m] GEMM 2 tiles of row tile m whose MMAs have read Z; a GEMM 1 tile two blocks
+//                  later overwrites those rows only once every one of them has.
+// CTAs take items in that order from a global counter and run them in order, and an item only
+// waits on items before it, all taken by resident CTAs (one CTA per SM, grid <= SMs): every wait
+// ends.  Every wait is bounded all the same (RA_ERR_TIMEOUT, then the CTA unwinds).
 //
-// CTA (256 threads, persistent, tiles t = blockIdx.x + i * gridDim.x, M-tiles fastest):
-//   warps 0-3  epilogue: thread = output row = TMEM lane; TMEM -> registers -> bias, GELU ->
-//              bf16 -> 16-byte global stores, 32 columns at a time;
-//   warp 4     TMA producer: per 64-wide K step, A 128 x 64 and B 256 x 64 into a 4-stage ring;
-//   warp 5     TMEM allocator + tcgen05.mma issuer (M = 128, N = 256, K = 16).
-// TMEM (512 columns): two 128 x 256 fp32 accumulators, so the epilogue of tile i overlaps the
-// MMAs of tile i + 1.
+// CTA (256 threads): warps 0-3 epilogue (thread = output row = TMEM lane), warp 4 TMA producer
+// (per 64-wide K step, A 128 x 64 and B 256 x 64 into a 4-stage ring, no multicast), warp 5 TMEM
+// allocator + tcgen05.mma issuer (M = 128, N = 256, K = 16, both operands K-major, 128-byte
+// swizzle).  TMEM: two 128 x 256 fp32 accumulators, so a tile's epilogue runs under the next
+// tile's MMAs.
 #pragma once
 #include "ra_sm100.cuh"
+#include "ra_work.cuh"
 
 namespace ra {
 namespace ffn {
@@ -40,60 +47,120 @@ struct Layout {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = NSTAGE * STAGE_BYTES;
   static constexpr int B_FULL = 0, B_EMPTY = NSTAGE, B_ACC_FULL = 2 * NSTAGE, B_ACC_EMPTY = B_ACC_FULL + 2,
-                       B_DRAIN = B_ACC_EMPTY + 2, NUM_BARS = B_DRAIN + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag
+                       B_DRAIN = B_ACC_EMPTY + 2, B_WQ_FULL = B_DRAIN + 1, B_WQ_EMPTY = B_WQ_FULL + 2,
+                       NUM_BARS = B_WQ_EMPTY + 2;
+  static constexpr uint32_t WQ_CONSUMERS = 1 + 4;         // MMA thread + one arrival per epilogue warp
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, item ring[2]
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;                // room to align the base to 1024 B
 };
 static_assert(Layout::ALLOC <= 232448, "shared memory");
 
 struct Params {
-  int K;                 // reduction length (multiple of BK)
-  int N;                 // output columns (multiple of 64)
-  int rows;              // rows of the block per batch entry (c)
-  int m_tiles_per_b;     // ceil(rows / BM)
-  int m_tiles;           // B * m_tiles_per_b
-  int n_tiles;           // ceil(N / BN)
-  int n_items;           // m_tiles * n_tiles
-  // A tile coordinates for (batch entry b, row tile tt, K offset k0):
-  //   (k0 % a_kdim, a_row0 + tt * BM, b * a_outer_per_b + k0 / a_kdim)
-  int a_kdim, a_row0, a_outer_per_b;
-  // output row of (b, r): b * c_rows_per_b + c_row0 + r, row-major with ldc columns
-  long long c_rows_per_b;
-  long long c_row0;
-  long long ldc;
-  const float* bias;     // [N]
-  __nv_bfloat16* c;
-  int gelu;              // 1: exact GELU after the bias
+  int S, H, Dh, c, h, f;
+  int r0, nblocks;       // ring blocks r0 .. r0 + nblocks - 1
+  int mt_per_b;          // row tiles per batch entry: ceil(c / BM)
+  int MT;                // row tiles per block: B * mt_per_b
+  int NT1, NT2;          // column tiles of GEMM 1 (f) and GEMM 2 (h)
+  int per_block;         // MT * (NT1 + NT2)
+  int n_items;           // nblocks * per_block
+  int work_slot;         // this launch's work counter
+  const float* b1;       // [f]
+  const float* b2;       // [h]
+  __nv_bfloat16* z;      // [2][B][c][f] hidden activations (one buffer when nblocks == 1)
+  __nv_bfloat16* y;      // [B][S][h]
+  unsigned* ready;       // [2][MT]
+  unsigned* consumed;    // [2][MT]
 };
 
-__device__ __forceinline__ void item_coords(int w, const Params& p, int& b, int& tt, int& nt) {
-  const int mt = w % p.m_tiles;
-  nt = w / p.m_tiles;
-  b = mt / p.m_tiles_per_b;
-  tt = mt - b * p.m_tiles_per_b;
+struct Tile {
+  int blk, u;            // block index in the launch, its Z buffer
+  int g;                 // 1: GEMM 1, 2: GEMM 2
+  int mt, nt, b, tt;     // row tile in the block, column tile, batch entry, row tile in the entry
+};
+
+__device__ __forceinline__ Tile decode(int w, const Params& p) {
+  Tile t;
+  t.blk = w / p.per_block;
+  int idx = w - t.blk * p.per_block;
+  t.u = t.blk & 1;
+  t.g = 1;
+  if (idx >= p.MT * p.NT1) {
+    idx -= p.MT * p.NT1;
+    t.g = 2;
+  }
+  t.mt = idx % p.MT;
+  t.nt = idx / p.MT;
+  t.b = t.mt / p.mt_per_b;
+  t.tt = t.mt - t.b * p.mt_per_b;
+  return t;
 }
 
 __device__ __forceinline__ float gelu_exact(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
 
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *ctr >= target (acquire): RA_ERR_TIMEOUT and false after the time limit or
+// once another warp of the CTA has given up.
+__device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target, volatile int* abort_flag) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if ((it & 63u) == 63u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > RA_WAIT_TIMEOUT_NS) break;
+    }
+    __nanosleep(64);
+  }
+  *abort_flag = 1;
+  record_status(RA_ERR_TIMEOUT);
+  return false;
+}
+
+__device__ __forceinline__ void signal_count(unsigned* ctr) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
 // ------------------------------------------------------------------ producer (1 thread)
-__device__ void producer(const CUtensorMap* tm_a, const CUtensorMap* tm_b, const Params& p, uint32_t sbase,
+__device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, const CUtensorMap* tm_z,
+                         const CUtensorMap* tm_w2, const Params& p, uint32_t sbase, volatile int* wq,
                          volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, issued = 0, issued_parity = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
-    int b, tt, nt;
-    item_coords(w, p, b, tt, nt);
-    for (int k0 = 0; k0 < p.K; k0 += BK) {
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  int w = work_fetch(p.work_slot);
+  for (;;) {
+    if (!ring.push(w, abort_flag)) { ok = false; break; }
+    if (w >= p.n_items) break;
+    const int w_next = work_fetch(p.work_slot);
+    const Tile t = decode(w, p);
+    const int r = p.r0 + t.blk;
+    const int K = t.g == 1 ? p.h : p.f;
+    if (t.g == 2) {   // every column tile of this row tile's hidden activation is stored
+      if (!wait_count(p.ready + t.u * p.MT + t.mt, static_cast<unsigned>(p.NT1 * (t.blk / 2 + 1)), abort_flag)) {
+        ok = false;
+        break;
+      }
+      fence_proxy_async_global();   // the generic-proxy stores of Z before these TMA reads
+    }
+    for (int k0 = 0; k0 < K; k0 += BK) {
       if (!mbar_wait(bar(L::B_EMPTY + stage), phase ^ 1u, abort_flag)) { ok = false; break; }
       const uint32_t st = sbase + stage * L::STAGE_BYTES;
       mbar_arrive_expect_tx(bar(L::B_FULL + stage), L::STAGE_BYTES);
-      tma_load_3d(tm_a, st, bar(L::B_FULL + stage), k0 % p.a_kdim, p.a_row0 + tt * BM,
-                  b * p.a_outer_per_b + k0 / p.a_kdim);
-      tma_load_3d(tm_b, st + L::A_BYTES, bar(L::B_FULL + stage), k0, nt * BN, 0);
+      if (t.g == 1) {
+        tma_load_3d(tm_x, st, bar(L::B_FULL + stage), k0 % p.Dh, r * p.c + t.tt * BM, t.b * p.H + k0 / p.Dh);
+        tma_load_3d(tm_w1, st + L::A_BYTES, bar(L::B_FULL + stage), k0, t.nt * BN, 0);
+      } else {
+        tma_load_3d(tm_z, st, bar(L::B_FULL + stage), k0, t.tt * BM, t.u * (p.MT / p.mt_per_b) + t.b);
+        tma_load_3d(tm_w2, st + L::A_BYTES, bar(L::B_FULL + stage), k0, t.nt * BN, 0);
+      }
       issued |= 1u << stage;
       issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
       if (++stage == NSTAGE) {
@@ -101,7 +168,10 @@ __device__ void producer(const CUtensorMap* tm_a, const CUtensorMap* tm_b, const
         phase ^= 1u;
       }
     }
+    if (!ok) break;
+    w = w_next;
   }
+  work_done(p.work_slot);
   if (!ok) {   // let every copy this CTA started land before the CTA can exit
     for (int s = 0; s < NSTAGE; ++s)
       if (issued & (1u << s)) drain_wait(bar(L::B_FULL + s), (issued_parity >> s) & 1u);
@@ -109,22 +179,27 @@ __device__ void producer(const CUtensorMap* tm_a, const CUtensorMap* tm_b, const
 }
 
 // ------------------------------------------------------------------ MMA issuer (1 thread)
-__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);   // A, B both K-major
   int stage = 0;
   uint32_t phase = 0;
-  uint32_t acc_phase[2] = {0, 0};
-  int j = 0;
-  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x, ++j) {
+  uint32_t acc_phases = 0;   // bit a: phase of accumulator a
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (int j = 0;; ++j) {
+    int w;
+    if (!ring.pop(w, abort_flag)) break;
+    if (w >= p.n_items) break;
+    const Tile t = decode(w, p);
+    const int K = t.g == 1 ? p.h : p.f;
     const int acc = j & 1;
-    if (!mbar_wait(bar(L::B_ACC_EMPTY + acc), acc_phase[acc] ^ 1u, abort_flag)) break;
-    acc_phase[acc] ^= 1u;
+    if (!mbar_wait(bar(L::B_ACC_EMPTY + acc), ((acc_phases >> acc) & 1u) ^ 1u, abort_flag)) break;
+    acc_phases ^= 1u << acc;
     tc_fence_after();
     const uint32_t d = tmem + acc * BN;
     bool ok = true;
-    for (int k0 = 0; k0 < p.K; k0 += BK) {
+    for (int k0 = 0; k0 < K; k0 += BK) {
       if (!mbar_wait(bar(L::B_FULL + stage), phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = sbase + stage * L::STAGE_BYTES, sb = sa + L::A_BYTES;
@@ -146,39 +221,61 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
 }
 
 // ------------------------------------------------------------------ epilogue (128 threads)
-__device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
+__device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   const int lane = threadIdx.x & 31;
   const int quarter = threadIdx.x >> 5;            // warps 0-3: TMEM lanes 32 * quarter + lane
   const int r = quarter * 32 + lane;               // row within the tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-  uint32_t acc_phase[2] = {0, 0};
-  int j = 0;
-  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x, ++j) {
+  uint32_t acc_phases = 0;   // bit a: phase of accumulator a
+  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
+  for (int j = 0;; ++j) {
+    int w = 0;
+    // warpgroup-uniform outcomes: the named barriers below need all four warps
+    if (!named_bar_and(1, 128, ring.pop_warp(w, abort_flag))) return;
+    if (w >= p.n_items) break;
+    const Tile t = decode(w, p);
     const int acc = j & 1;
-    if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_ACC_FULL + acc), acc_phase[acc], abort_flag))) return;
-    acc_phase[acc] ^= 1u;
+    if (!named_bar_and(1, 128, mbar_wait(bar(L::B_ACC_FULL + acc), (acc_phases >> acc) & 1u, abort_flag))) return;
+    acc_phases ^= 1u << acc;
     tc_fence_after();
-    int b, tt, nt;
-    item_coords(w, p, b, tt, nt);
-    const int row_in_block = tt * BM + r;
-    const bool row_ok = row_in_block < p.rows;
-    __nv_bfloat16* crow = p.c + (static_cast<long long>(b) * p.c_rows_per_b + p.c_row0 + row_in_block) * p.ldc;
-    const int n_base = nt * BN;
+    const int row_in_block = t.tt * BM + r;
+    const bool row_ok = row_in_block < p.c;
+    __nv_bfloat16* crow;
+    const float* bias;
+    int N;
+    if (t.g == 1) {
+      // Z_u rows of this row tile are overwritten only once the GEMM 2 tiles of the block two
+      // before have read them
+      bool go = true;
+      if (t.blk >= 2 && threadIdx.x == 0)
+        go = wait_count(p.consumed + t.u * p.MT + t.mt, static_cast<unsigned>(p.NT2 * (t.blk / 2)), abort_flag);
+      if (!named_bar_and(1, 128, go)) return;
+      crow = p.z + ((static_cast<long long>(t.u) * (p.MT / p.mt_per_b) + t.b) * p.c + row_in_block) * p.f;
+      bias = p.b1;
+      N = p.f;
+    } else {
+      // this tile's MMAs have read its Z rows: they may be overwritten
+      if (threadIdx.x == 0) signal_count(p.consumed + t.u * p.MT + t.mt);
+      crow = p.y + (static_cast<long long>(t.b) * p.S + static_cast<long long>(p.r0 + t.blk) * p.c + row_in_block) * p.h;
+      bias = p.b2;
+      N = p.h;
+    }
+    const int n_base = t.nt * BN;
 #pragma unroll 1
     for (int ch = 0; ch < BN / 32; ++ch) {
       const int n0 = n_base + 32 * ch;
-      if (n0 >= p.N) break;   // uniform: N is a multiple of 64
+      if (n0 >= N) break;   // uniform: N is a multiple of 64
       uint32_t v[32];
       tmem_ld32(lane_base + acc * BN + 32 * ch, v);
       tmem_ld_wait();
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float2 bb = __ldg(reinterpret_cast<const float2*>(p.bias + n0) + i);
+        const float2 bb = __ldg(reinterpret_cast<const float2*>(bias + n0) + i);
         float x0 = __uint_as_float(v[2 * i]) + bb.x, x1 = __uint_as_float(v[2 * i + 1]) + bb.y;
-        if (p.gelu) {
+        if (t.g == 1) {
           x0 = gelu_exact(x0);
           x1 = gelu_exact(x1);
         }
@@ -193,23 +290,32 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatil
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(L::B_ACC_EMPTY + acc));   // 4 arrivals: the accumulator is free
+    if (t.g == 1) {   // publish this tile's Z columns to the GEMM 2 tiles of its row tile
+      fence_proxy_async_global();   // for the TMA (async proxy) reads that follow elsewhere
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 0) signal_count(p.ready + t.u * p.MT + t.mt);
+    }
   }
 }
 
 // ------------------------------------------------------------------ kernel
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const Params p) {
+    ffn_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w1,
+               const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_w2, const Params p) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  volatile int* wq = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       const bool acc_empty = i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1;
-      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 4 : 1);
+      const bool wq_empty = i == L::B_WQ_EMPTY || i == L::B_WQ_EMPTY + 1;
+      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 4 : (wq_empty ? L::WQ_CONSUMERS : 1));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -219,8 +325,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_relinquish();
   }
   if (warp == WARP_TMA && (threadIdx.x & 31) == 0) {
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w1);
+    tma_prefetch_desc(&tm_z);
+    tma_prefetch_desc(&tm_w2);
   }
   tc_fence_before();
   __syncthreads();
@@ -228,12 +336,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp < 4) {
-    epilogue(p, sbase, tmem, abort_flag);
+    epilogue(p, sbase, tmem, wq, abort_flag);
   } else if (warp == WARP_TMA) {
-    if ((threadIdx.x & 31) == 0) producer(&tm_a, &tm_b, p, sbase, abort_flag);
+    if ((threadIdx.x & 31) == 0) producer(&tm_x, &tm_w1, &tm_z, &tm_w2, p, sbase, wq, abort_flag);
     __syncwarp();
   } else if (warp == WARP_MMA) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, abort_flag);
+    if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, wq, abort_flag);
     __syncwarp();
   }
 

@@ -665,8 +665,21 @@ int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
 // --- blockwise feedforward after attention ------------------------------------------------
 namespace {
 
-size_t ffn_workspace(int B, int S, int D, int f) {
-  return align256(static_cast<size_t>(B) * (S / D) * f * 2);
+// Workspace: two block-sized hidden activations (bf16 [2][B][c][f]) then the per-row-tile
+// dependency counters ([2][MT] ready, [2][MT] consumed), each region 256-byte aligned.
+struct FfnWorkspace {
+  size_t z_bytes, ctr_bytes, total;
+  int mt;
+};
+
+FfnWorkspace ffn_workspace(int B, int S, int D, int f) {
+  FfnWorkspace w;
+  const int c = S / D;
+  w.mt = B * ((c + ra::ffn::BM - 1) / ra::ffn::BM);
+  w.z_bytes = align256(2 * static_cast<size_t>(B) * c * f * 2);
+  w.ctr_bytes = align256(static_cast<size_t>(4) * w.mt * sizeof(unsigned));
+  w.total = w.z_bytes + w.ctr_bytes;
+  return w;
 }
 
 // Arguments shared by the two feedforward entry points; RA_OK when usable.
@@ -685,72 +698,61 @@ int ffn_check(const void* o, int B, int H, int S, int Dh, int D, const void* w1,
                           static_cast<const void*>(y)})
     if (!aligned16(ptr)) return RA_ERR_ALIGN;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      workspace_bytes < ffn_workspace(B, S, D, f))
+      workspace_bytes < ffn_workspace(B, S, D, f).total)
     return RA_ERR_WORKSPACE;
   return RA_OK;
 }
 
-int ffn_gemm(DevInfo* di, const CUtensorMap& ma, const CUtensorMap& mb, ra::ffn::Params& p, cudaStream_t stream) {
+// Feedforward of ring blocks r0 .. r0 + nblocks - 1 in one persistent launch (after clearing the
+// dependency counters on the stream).
+int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nblocks, const void* w1, const float* b1,
+            const void* w2, const float* b2, int f, void* y, void* workspace, cudaStream_t stream) {
   namespace rf = ra::ffn;
-  p.m_tiles_per_b = (p.rows + rf::BM - 1) / rf::BM;
-  p.n_tiles = (p.N + rf::BN - 1) / rf::BN;
-  const long long items = static_cast<long long>(p.m_tiles) * p.n_tiles;
-  if (items > INT_MAX) return RA_ERR_SHAPE;
-  p.n_items = static_cast<int>(items);
-  constexpr int smem = rf::Layout::ALLOC;
-  if (!di->ffn_attr) {
-    const cudaError_t e = cudaFuncSetAttribute(rf::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(ffn smem)");
-    di->ffn_attr = true;
-  }
-  const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
-  rf::gemm_kernel<<<grid, rf::NUM_THREADS, smem, stream>>>(ma, mb, p);
-  return launch_status();
-}
-
-// Feedforward of ring block r: GEMM 1 (attention output -> hidden activation Z in the
-// workspace, bias + GELU) then GEMM 2 (Z -> y rows of the block, bias).
-int ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r, const void* w1, const float* b1,
-              const void* w2, const float* b2, int f, void* y, void* workspace, cudaStream_t stream) {
   int st = RA_OK;
   DevInfo* di = dev_info(&st);
   if (!di) return st;
-  const int c = S / D;
-  const int h = H * Dh;
-  ra::ffn::Params p1{};
-  p1.K = h;
-  p1.N = f;
-  p1.rows = c;
-  p1.m_tiles = B * ((c + ra::ffn::BM - 1) / ra::ffn::BM);
-  p1.a_kdim = Dh;
-  p1.a_row0 = r * c;
-  p1.a_outer_per_b = H;
-  p1.c_rows_per_b = c;
-  p1.c_row0 = 0;
-  p1.ldc = f;
-  p1.bias = b1;
-  p1.c = static_cast<__nv_bfloat16*>(workspace);
-  p1.gelu = 1;
-  CUtensorMap ma, mb;
-  if ((st = make_map(&ma, o, static_cast<long long>(B) * H, S, Dh, ra::ffn::BM)) != RA_OK) return st;
-  if ((st = make_map(&mb, w1, 1, f, h, ra::ffn::BN)) != RA_OK) return st;
-  if ((st = ffn_gemm(di, ma, mb, p1, stream)) != RA_OK) return st;
-
-  ra::ffn::Params p2 = p1;
-  p2.K = f;
-  p2.N = h;
-  p2.a_kdim = f;
-  p2.a_row0 = 0;
-  p2.a_outer_per_b = 1;
-  p2.c_rows_per_b = S;
-  p2.c_row0 = static_cast<long long>(r) * c;
-  p2.ldc = h;
-  p2.bias = b2;
-  p2.c = static_cast<__nv_bfloat16*>(y);
-  p2.gelu = 0;
-  if ((st = make_map(&ma, workspace, B, c, f, ra::ffn::BM)) != RA_OK) return st;
-  if ((st = make_map(&mb, w2, 1, h, f, ra::ffn::BN)) != RA_OK) return st;
-  return ffn_gemm(di, ma, mb, p2, stream);
+  const FfnWorkspace ws = ffn_workspace(B, S, D, f);
+  rf::Params p{};
+  p.S = S;
+  p.H = H;
+  p.Dh = Dh;
+  p.c = S / D;
+  p.h = H * Dh;
+  p.f = f;
+  p.r0 = r0;
+  p.nblocks = nblocks;
+  p.mt_per_b = (p.c + rf::BM - 1) / rf::BM;
+  p.MT = ws.mt;
+  p.NT1 = (f + rf::BN - 1) / rf::BN;
+  p.NT2 = (p.h + rf::BN - 1) / rf::BN;
+  const long long per_block = static_cast<long long>(p.MT) * (p.NT1 + p.NT2);
+  if (per_block * nblocks > INT_MAX) return RA_ERR_SHAPE;
+  p.per_block = static_cast<int>(per_block);
+  p.n_items = static_cast<int>(per_block * nblocks);
+  p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
+  p.b1 = b1;
+  p.b2 = b2;
+  p.z = static_cast<__nv_bfloat16*>(workspace);
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ready = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + ws.z_bytes);
+  p.consumed = p.ready + 2 * p.MT;
+  CUtensorMap mx, mw1, mz, mw2;
+  if ((st = make_map(&mx, o, static_cast<long long>(B) * H, S, Dh, rf::BM)) != RA_OK) return st;
+  if ((st = make_map(&mw1, w1, 1, f, p.h, rf::BN)) != RA_OK) return st;
+  if ((st = make_map(&mz, workspace, 2ll * B, p.c, f, rf::BM)) != RA_OK) return st;
+  if ((st = make_map(&mw2, w2, 1, p.h, f, rf::BN)) != RA_OK) return st;
+  const cudaError_t me = cudaMemsetAsync(p.ready, 0, 4 * static_cast<size_t>(p.MT) * sizeof(unsigned), stream);
+  if (me != cudaSuccess) return cuda_fail(static_cast<int>(me), "cudaMemsetAsync(ffn counters)");
+  constexpr int smem = rf::Layout::ALLOC;
+  if (!di->ffn_attr) {
+    const cudaError_t e = cudaFuncSetAttribute(rf::ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(ffn smem)");
+    di->ffn_attr = true;
+  }
+  // one CTA per SM at most, all resident: an item waits only on items taken before it
+  const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
+  rf::ffn_kernel<<<grid, rf::NUM_THREADS, smem, stream>>>(mx, mw1, mz, mw2, p);
+  return launch_status();
 }
 
 }  // namespace
@@ -759,7 +761,7 @@ extern "C" {
 
 size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f) {
   if (B <= 0 || S <= 0 || D <= 0 || D > S || S % D != 0 || f <= 0) return 0;
-  return ffn_workspace(B, S, D, f);
+  return ffn_workspace(B, S, D, f).total;
 }
 
 int ring_attn_ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r, const void* w1, const float* b1,
@@ -768,7 +770,7 @@ int ring_attn_ffn_block(const void* o, int B, int H, int S, int Dh, int D, int r
   int st = ffn_check(o, B, H, S, Dh, D, w1, b1, w2, b2, f, y, workspace, workspace_bytes);
   if (st != RA_OK) return st;
   if (r < 0 || r >= D) return RA_ERR_ARG;
-  return ffn_block(o, B, H, S, Dh, D, r, w1, b1, w2, b2, f, y, workspace, static_cast<cudaStream_t>(stream));
+  return ffn_run(o, B, H, S, Dh, D, r, 1, w1, b1, w2, b2, f, y, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int ring_attn_ffn_fwd(const void* o, int B, int H, int S, int Dh, int D, const void* w1, const float* b1,
@@ -776,11 +778,7 @@ int ring_attn_ffn_fwd(const void* o, int B, int H, int S, int Dh, int D, const v
                       ra_stream stream) {
   int st = ffn_check(o, B, H, S, Dh, D, w1, b1, w2, b2, f, y, workspace, workspace_bytes);
   if (st != RA_OK) return st;
-  for (int r = 0; r < D; ++r) {
-    st = ffn_block(o, B, H, S, Dh, D, r, w1, b1, w2, b2, f, y, workspace, static_cast<cudaStream_t>(stream));
-    if (st != RA_OK) return st;
-  }
-  return RA_OK;
+  return ffn_run(o, B, H, S, Dh, D, 0, D, w1, b1, w2, b2, f, y, workspace, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
