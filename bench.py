@@ -101,7 +101,7 @@ def _peaks():
 KERNEL_SOURCES = {
     "fwd_kernel": ("fwd_sm100.cuh", "ra_sm100.cuh", "ra_schedule.h", "ra_work.cuh", "ring_attn.cu"),
     "bwd_kernel": ("bwd_sm100.cuh", "ra_sm100.cuh", "ra_schedule.h", "ra_work.cuh", "ring_attn.cu"),
-    "gemm_kernel": ("ffn_sm100.cuh", "ra_sm100.cuh", "ring_attn.cu"),
+    "ffn_kernel": ("ffn_sm100.cuh", "ra_sm100.cuh", "ra_work.cuh", "ring_attn.cu"),
 }
 
 
@@ -369,7 +369,7 @@ def time_ffn_leg(w: Workload, dev, stream, warmup: int):
     torch.cuda.empty_cache()
     return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "frac": flops / (ms * 1e-3) / 1e12 / peak,
             "peak": peak, "peak_source": f"{src} {'sustained' if sustained else 'burst'} bf16 dense",
-            "launches_timed": n, "timed_s": t_wall, "traffic": _traffic("gemm_kernel", "s16k_ffn"),
+            "launches_timed": n, "timed_s": t_wall, "traffic": _traffic("ffn_kernel", "s16k_ffn"),
             "config": {"B": w.B, "S": w.S, "h": h, "f": f, "D": w.D, "c": w.c, "flops": flops,
                        "activation_bytes": 2 * w.B * w.c * f, "weights": f"seeded, seed {w.seed + 77}"},
             "clocks": clocks.summary()}
