@@ -400,7 +400,7 @@ def run_ours(args, w: Workload):
         split_ws = torch.empty(ra.fwd_split_workspace_bytes(w.B, w.H, w.S, w.Dh, args.parts), dtype=torch.uint8,
                                device=dev)
     stream = torch.cuda.current_stream(dev)
-    flush_needed = "flushed" in _config(w, args)["l2"]
+    flush_needed = _config(w, args)["l2"].startswith("L2 flushed")
     flush_buf = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev) if flush_needed else None
 
     def step(evs=None, xin=None, res=None, st=None):
