@@ -230,7 +230,7 @@ RA_API size_t ring_attn_bwd_noalloc_max_bytes(void);
 /*
  * ring_attn_ffn_workspace_size -- bytes of device workspace the blockwise feedforward needs: two
  * ring blocks' hidden activations, bf16 [2][B][S / D][f] (block r + 1's first product runs while
- * block r's second drains), then 4 * B * ceil((S / D) / 128) 32-bit dependency counters, each
+ * block r's second drains), then 4 * B * ceil((S / D) / 256) 32-bit dependency counters, each
  * region rounded up to 256 bytes.  Independent of D for a given block size: the activation alive
  * is two blocks', never the sequence's.  Returns 0 for invalid sizes.
  */
@@ -256,9 +256,10 @@ RA_API size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f);
  *             aligned: the hidden activation gelu(x W1^T + b1), rounded to bf16 (the activation
  *             the pages' memory count stores), and the dependency counters; overwritten by every
  *             call.
- * A memset of the counters and one persistent launch on `stream`: tcgen05 tiles of both
- * products (bias + GELU epilogue, then bias epilogue), float32 accumulation; a tile of the
- * second product starts once the first product's tiles of its rows are stored.  Pointers
+ * A memset of the counters and one persistent launch of CTA pairs (clusters of two CTAs on
+ * neighbouring SMs) on `stream`: tcgen05 tiles of both products (bias + GELU epilogue, then bias
+ * epilogue), float32 accumulation; a tile of the second product starts once the first product's
+ * tiles of its rows are stored.  Pointers
  * 16-byte aligned.  Calls that overlap on the GPU must not share a workspace.  Errors:
  * RA_ERR_ARG (null pointer, f <= 0, r out of range), RA_ERR_SHAPE (S % D, Dh, f % 64, sizes),
  * RA_ERR_ALIGN, RA_ERR_WORKSPACE, RA_ERR_CUDA; RA_ERR_TIMEOUT in the device status word if a

@@ -23,34 +23,40 @@
 // waits on items before it, all taken by resident CTAs (one CTA per SM, grid <= SMs): every wait
 // ends.  Every wait is bounded all the same (RA_ERR_TIMEOUT, then the CTA unwinds).
 //
-// CTA (256 threads): warps 0-3 epilogue (thread = output row = TMEM lane), warp 4 TMA producer
-// (per 64-wide K step, A 128 x 64 and B 256 x 64 into a 4-stage ring, no multicast), warp 5 TMEM
-// allocator + tcgen05.mma issuer (M = 128, N = 256, K = 16, both operands K-major, 128-byte
-// swizzle).  TMEM: two 128 x 256 fp32 accumulators, so a tile's epilogue runs under the next
-// tile's MMAs.
+// A CTA pair (cluster of 2, tcgen05 cta_group::2) computes each 256-row x 256-column tile: each
+// CTA loads its own 128 rows of A and its own 128 of the tile's 256 B rows (weight rows), and one
+// M = 256, N = 256 MMA per 16-wide K step runs on both SMs, so an SM brings in 32 KiB per 64-wide K
+// step for 512 tensor cycles (64 B per clock, against 96 for a single CTA with 128 x 256 tiles).
+// Loads of both CTAs complete on the even CTA's barriers; the even CTA's one MMA thread issues
+// every MMA and commits to barriers in both CTAs.  Tiles are taken round robin by CTA pair.
+// CTA (256 threads): warps 0-3 epilogue (thread = output row = TMEM lane; the even CTA holds rows
+// 0-127 of the tile, the odd one rows 128-255), warp 4 TMA producer (6-stage ring of 32 KiB, no
+// multicast), warp 5 TMEM allocation (both CTAs) and, in the even CTA, the tcgen05.mma issue.
+// TMEM per CTA: two 128 x 256 fp32 accumulators, so a tile's epilogue runs under the next tile's
+// MMAs.
 #pragma once
 #include "ra_sm100.cuh"
-#include "ra_work.cuh"
 
 namespace ra {
 namespace ffn {
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int NSTAGE = 4;
+constexpr int BM = 256, BN = 256, BK = 64;   // tile of a CTA pair
+constexpr int HALF = 128;                     // rows of A and of B per CTA
+constexpr int NSTAGE = 6;
 constexpr int NUM_THREADS = 256;
 constexpr int WARP_TMA = 4, WARP_MMA = 5;
 constexpr uint32_t TMEM_COLS = 512;
 
 struct Layout {
-  static constexpr int A_BYTES = BM * BK * 2;            // 16 KB, 128 rows x 128 B
-  static constexpr int B_BYTES = BN * BK * 2;            // 32 KB, 256 rows x 128 B
+  static constexpr int A_BYTES = HALF * BK * 2;          // 16 KB: this CTA's 128 rows x 128 B
+  static constexpr int B_BYTES = HALF * BK * 2;          // 16 KB: this CTA's 128 of the 256 B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = NSTAGE * STAGE_BYTES;
+  // FULL: used in the even CTA (both CTAs' loads complete on it); EMPTY, ACC_FULL: in both CTAs
+  // (the even CTA's MMA commits to both); ACC_EMPTY: in the even CTA (4 warps of each CTA arrive)
   static constexpr int B_FULL = 0, B_EMPTY = NSTAGE, B_ACC_FULL = 2 * NSTAGE, B_ACC_EMPTY = B_ACC_FULL + 2,
-                       B_DRAIN = B_ACC_EMPTY + 2, B_WQ_FULL = B_DRAIN + 1, B_WQ_EMPTY = B_WQ_FULL + 2,
-                       NUM_BARS = B_WQ_EMPTY + 2;
-  static constexpr uint32_t WQ_CONSUMERS = 1 + 4;         // MMA thread + one arrival per epilogue warp
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, item ring[2]
+                       B_DRAIN = B_ACC_EMPTY + 2, NUM_BARS = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;                // room to align the base to 1024 B
 };
@@ -59,12 +65,11 @@ static_assert(Layout::ALLOC <= 232448, "shared memory");
 struct Params {
   int S, H, Dh, c, h, f;
   int r0, nblocks;       // ring blocks r0 .. r0 + nblocks - 1
-  int mt_per_b;          // row tiles per batch entry: ceil(c / BM)
+  int mt_per_b;          // row tiles per batch entry: ceil(c / BM)  (BM = 256, a CTA pair)
   int MT;                // row tiles per block: B * mt_per_b
   int NT1, NT2;          // column tiles of GEMM 1 (f) and GEMM 2 (h)
   int per_block;         // MT * (NT1 + NT2)
   int n_items;           // nblocks * per_block
-  int work_slot;         // this launch's work counter
   const float* b1;       // [f]
   const float* b2;       // [h]
   __nv_bfloat16* z;      // [2][B][c][f] hidden activations (one buffer when nblocks == 1)
@@ -125,26 +130,65 @@ __device__ __forceinline__ void signal_count(unsigned* ctr) {
   asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 
-// ------------------------------------------------------------------ producer (1 thread)
+// ------------------------------------------------------------------ CTA-pair primitives
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// 3-D tile load into this CTA's shared memory whose completion is counted on a barrier of the
+// pair (the even CTA's): the cta_group::2 form, no multicast.
+__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap* map, uint32_t dst, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar_cluster` (a barrier of either CTA) once this thread's pair MMAs complete.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+// ------------------------------------------------------------------ producer (1 thread per CTA)
 __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, const CUtensorMap* tm_z,
-                         const CUtensorMap* tm_w2, const Params& p, uint32_t sbase, volatile int* wq,
-                         volatile int* abort_flag) {
+                         const CUtensorMap* tm_w2, const Params& p, uint32_t sbase, uint32_t rank, int pair,
+                         int n_pairs, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, issued = 0, issued_parity = 0;
   bool ok = true;
-  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
-  int w = work_fetch(p.work_slot);
-  for (;;) {
-    if (!ring.push(w, abort_flag)) { ok = false; break; }
-    if (w >= p.n_items) break;
-    const int w_next = work_fetch(p.work_slot);
+  for (int w = pair; w < p.n_items && ok; w += n_pairs) {
     const Tile t = decode(w, p);
     const int r = p.r0 + t.blk;
     const int K = t.g == 1 ? p.h : p.f;
-    if (t.g == 2) {   // every column tile of this row tile's hidden activation is stored
-      if (!wait_count(p.ready + t.u * p.MT + t.mt, static_cast<unsigned>(p.NT1 * (t.blk / 2 + 1)), abort_flag)) {
+    const int row = t.tt * BM + rank * HALF;   // this CTA's rows of the tile, within the batch entry
+    if (t.g == 2) {   // every column tile of this row tile's hidden activation is stored (both CTAs)
+      if (!wait_count(p.ready + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT1 * (t.blk / 2 + 1)), abort_flag)) {
         ok = false;
         break;
       }
@@ -153,13 +197,14 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, cons
     for (int k0 = 0; k0 < K; k0 += BK) {
       if (!mbar_wait(bar(L::B_EMPTY + stage), phase ^ 1u, abort_flag)) { ok = false; break; }
       const uint32_t st = sbase + stage * L::STAGE_BYTES;
-      mbar_arrive_expect_tx(bar(L::B_FULL + stage), L::STAGE_BYTES);
+      const uint32_t full = map_to_rank(bar(L::B_FULL + stage), 0);   // the even CTA's barrier
+      if (rank == 0) mbar_arrive_expect_tx(bar(L::B_FULL + stage), 2 * L::STAGE_BYTES);   // both CTAs' bytes
       if (t.g == 1) {
-        tma_load_3d(tm_x, st, bar(L::B_FULL + stage), k0 % p.Dh, r * p.c + t.tt * BM, t.b * p.H + k0 / p.Dh);
-        tma_load_3d(tm_w1, st + L::A_BYTES, bar(L::B_FULL + stage), k0, t.nt * BN, 0);
+        tma_load_3d_pair(tm_x, st, full, k0 % p.Dh, r * p.c + row, t.b * p.H + k0 / p.Dh);
+        tma_load_3d_pair(tm_w1, st + L::A_BYTES, full, k0, t.nt * BN + rank * HALF, 0);
       } else {
-        tma_load_3d(tm_z, st, bar(L::B_FULL + stage), k0, t.tt * BM, t.u * (p.MT / p.mt_per_b) + t.b);
-        tma_load_3d(tm_w2, st + L::A_BYTES, bar(L::B_FULL + stage), k0, t.nt * BN, 0);
+        tma_load_3d_pair(tm_z, st, full, k0, row, t.u * (p.MT / p.mt_per_b) + t.b);
+        tma_load_3d_pair(tm_w2, st + L::A_BYTES, full, k0, t.nt * BN + rank * HALF, 0);
       }
       issued |= 1u << stage;
       issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -168,29 +213,28 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, cons
         phase ^= 1u;
       }
     }
-    if (!ok) break;
-    w = w_next;
   }
-  work_done(p.work_slot);
-  if (!ok) {   // let every copy this CTA started land before the CTA can exit
+  if (!ok && rank == 0) {   // let every copy the pair started land (they count on these barriers)
     for (int s = 0; s < NSTAGE; ++s)
       if (issued & (1u << s)) drain_wait(bar(L::B_FULL + s), (issued_parity >> s) & 1u);
   }
 }
 
-// ------------------------------------------------------------------ MMA issuer (1 thread)
-__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
+// ------------------------------------------------------------------ MMA issuer (1 thread, even CTA)
+__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, int pair, int n_pairs,
+                           volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);   // A, B both K-major
+  auto both = [&](int i) {   // commit to barrier i of each CTA
+    tc_commit_pair(map_to_rank(bar(i), 0));
+    tc_commit_pair(map_to_rank(bar(i), 1));
+  };
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);   // M = 256 over the pair, A, B K-major
   int stage = 0;
   uint32_t phase = 0;
   uint32_t acc_phases = 0;   // bit a: phase of accumulator a
-  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
-  for (int j = 0;; ++j) {
-    int w;
-    if (!ring.pop(w, abort_flag)) break;
-    if (w >= p.n_items) break;
+  int j = 0;
+  for (int w = pair; w < p.n_items; w += n_pairs, ++j) {
     const Tile t = decode(w, p);
     const int K = t.g == 1 ? p.h : p.f;
     const int acc = j & 1;
@@ -205,38 +249,36 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
       const uint32_t sa = sbase + stage * L::STAGE_BYTES, sb = sa + L::A_BYTES;
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk)
-        umma_ss(d, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024), IDESC,
-                (k0 > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(bar(L::B_EMPTY + stage));   // the stage is free once these MMAs have read it
+        umma_ss_pair(d, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024), IDESC,
+                     (k0 > 0 || kk > 0) ? 1u : 0u);
+      both(L::B_EMPTY + stage);   // the stage is free in both CTAs once these MMAs have read it
       if (++stage == NSTAGE) {
         stage = 0;
         phase ^= 1u;
       }
     }
     if (!ok) break;
-    tc_commit(bar(L::B_ACC_FULL + acc));
+    both(L::B_ACC_FULL + acc);
   }
-  tc_commit(bar(L::B_DRAIN));   // every MMA issued so far has completed before TMEM is released
+  tc_commit_pair(map_to_rank(bar(L::B_DRAIN), 0));   // every MMA issued so far has completed
   drain_wait(bar(L::B_DRAIN), 0);
 }
 
-// ------------------------------------------------------------------ epilogue (128 threads)
-__device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* wq, volatile int* abort_flag) {
+// ------------------------------------------------------------------ epilogue (128 threads per CTA)
+__device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_t rank, int pair, int n_pairs,
+                         volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   const int lane = threadIdx.x & 31;
   const int quarter = threadIdx.x >> 5;            // warps 0-3: TMEM lanes 32 * quarter + lane
-  const int r = quarter * 32 + lane;               // row within the tile
+  const int r = static_cast<int>(rank) * HALF + quarter * 32 + lane;   // row within the pair's tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
   uint32_t acc_phases = 0;   // bit a: phase of accumulator a
-  ItemRing ring{bar(L::B_WQ_FULL), bar(L::B_WQ_EMPTY), wq};
-  for (int j = 0;; ++j) {
-    int w = 0;
-    // warpgroup-uniform outcomes: the named barriers below need all four warps
-    if (!named_bar_and(1, 128, ring.pop_warp(w, abort_flag))) return;
-    if (w >= p.n_items) break;
+  int j = 0;
+  for (int w = pair; w < p.n_items; w += n_pairs, ++j) {
     const Tile t = decode(w, p);
     const int acc = j & 1;
+    // uniform outcomes across the four warps: the named barriers below need all of them
     if (!named_bar_and(1, 128, mbar_wait(bar(L::B_ACC_FULL + acc), (acc_phases >> acc) & 1u, abort_flag))) return;
     acc_phases ^= 1u << acc;
     tc_fence_after();
@@ -250,13 +292,13 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatil
       // before have read them
       bool go = true;
       if (t.blk >= 2 && threadIdx.x == 0)
-        go = wait_count(p.consumed + t.u * p.MT + t.mt, static_cast<unsigned>(p.NT2 * (t.blk / 2)), abort_flag);
+        go = wait_count(p.consumed + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT2 * (t.blk / 2)), abort_flag);
       if (!named_bar_and(1, 128, go)) return;
       crow = p.z + ((static_cast<long long>(t.u) * (p.MT / p.mt_per_b) + t.b) * p.c + row_in_block) * p.f;
       bias = p.b1;
       N = p.f;
     } else {
-      // this tile's MMAs have read its Z rows: they may be overwritten
+      // this tile's MMAs have read its Z rows in this CTA: they may be overwritten
       if (threadIdx.x == 0) signal_count(p.consumed + t.u * p.MT + t.mt);
       crow = p.y + (static_cast<long long>(t.b) * p.S + static_cast<long long>(p.r0 + t.blk) * p.c + row_in_block) * p.h;
       bias = p.b2;
@@ -289,8 +331,9 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatil
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar(L::B_ACC_EMPTY + acc));   // 4 arrivals: the accumulator is free
-    if (t.g == 1) {   // publish this tile's Z columns to the GEMM 2 tiles of its row tile
+    // 8 arrivals on the even CTA's barrier (4 warps of each CTA): the accumulator is free
+    if (lane == 0) mbar_arrive_cluster(map_to_rank(bar(L::B_ACC_EMPTY + acc), 0));
+    if (t.g == 1) {   // publish this CTA's half of the tile's Z columns
       fence_proxy_async_global();   // for the TMA (async proxy) reads that follow elsewhere
       __threadfence();
       named_bar_sync(1, 128);
@@ -299,8 +342,8 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, volatil
   }
 }
 
-// ------------------------------------------------------------------ kernel
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// ------------------------------------------------------------------ kernel (clusters of 2 CTAs)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ffn_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w1,
                const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_w2, const Params p) {
   using L = Layout;
@@ -309,20 +352,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
-  volatile int* wq = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
   const int warp = threadIdx.x >> 5;
+  const uint32_t rank = cluster_rank();
+  const int pair = static_cast<int>(blockIdx.x >> 1), n_pairs = static_cast<int>(gridDim.x >> 1);
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       const bool acc_empty = i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1;
-      const bool wq_empty = i == L::B_WQ_EMPTY || i == L::B_WQ_EMPTY + 1;
-      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 4 : (wq_empty ? L::WQ_CONSUMERS : 1));
+      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 8 : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == WARP_MMA) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
-    tmem_relinquish();
+  if (warp == WARP_MMA) {   // both CTAs, the same warp: the pair's TMEM
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   if (warp == WARP_TMA && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_x);
@@ -332,25 +377,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // both CTAs' barriers are initialised before either CTA touches the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
   if (warp < 4) {
-    epilogue(p, sbase, tmem, wq, abort_flag);
+    epilogue(p, sbase, tmem, rank, pair, n_pairs, abort_flag);
   } else if (warp == WARP_TMA) {
-    if ((threadIdx.x & 31) == 0) producer(&tm_x, &tm_w1, &tm_z, &tm_w2, p, sbase, wq, abort_flag);
+    if ((threadIdx.x & 31) == 0) producer(&tm_x, &tm_w1, &tm_z, &tm_w2, p, sbase, rank, pair, n_pairs, abort_flag);
     __syncwarp();
   } else if (warp == WARP_MMA) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, wq, abort_flag);
+    if (rank == 0 && (threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, pair, n_pairs, abort_flag);
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // the pair's MMAs have drained and both epilogues are done with TMEM
   if (warp == WARP_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
+  cluster_sync();   // neither CTA leaves while the other may still address its shared memory
 }
 
 }  // namespace ffn

@@ -729,7 +729,6 @@ int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nbloc
   if (per_block * nblocks > INT_MAX) return RA_ERR_SHAPE;
   p.per_block = static_cast<int>(per_block);
   p.n_items = static_cast<int>(per_block * nblocks);
-  p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.b1 = b1;
   p.b2 = b2;
   p.z = static_cast<__nv_bfloat16*>(workspace);
@@ -737,10 +736,11 @@ int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nbloc
   p.ready = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + ws.z_bytes);
   p.consumed = p.ready + 2 * p.MT;
   CUtensorMap mx, mw1, mz, mw2;
-  if ((st = make_map(&mx, o, static_cast<long long>(B) * H, S, Dh, rf::BM)) != RA_OK) return st;
-  if ((st = make_map(&mw1, w1, 1, f, p.h, rf::BN)) != RA_OK) return st;
-  if ((st = make_map(&mz, workspace, 2ll * B, p.c, f, rf::BM)) != RA_OK) return st;
-  if ((st = make_map(&mw2, w2, 1, p.h, f, rf::BN)) != RA_OK) return st;
+  // each CTA of a pair loads 128 rows of A and 128 of the tile's 256 B rows per K step
+  if ((st = make_map(&mx, o, static_cast<long long>(B) * H, S, Dh, rf::HALF)) != RA_OK) return st;
+  if ((st = make_map(&mw1, w1, 1, f, p.h, rf::HALF)) != RA_OK) return st;
+  if ((st = make_map(&mz, workspace, 2ll * B, p.c, f, rf::HALF)) != RA_OK) return st;
+  if ((st = make_map(&mw2, w2, 1, p.h, f, rf::HALF)) != RA_OK) return st;
   const cudaError_t me = cudaMemsetAsync(p.ready, 0, 4 * static_cast<size_t>(p.MT) * sizeof(unsigned), stream);
   if (me != cudaSuccess) return cuda_fail(static_cast<int>(me), "cudaMemsetAsync(ffn counters)");
   constexpr int smem = rf::Layout::ALLOC;
@@ -749,9 +749,12 @@ int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nbloc
     if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(ffn smem)");
     di->ffn_attr = true;
   }
-  // one CTA per SM at most, all resident: an item waits only on items taken before it
-  const int grid = p.n_items < di->sm_count ? p.n_items : di->sm_count;
-  rf::ffn_kernel<<<grid, rf::NUM_THREADS, smem, stream>>>(mx, mw1, mz, mw2, p);
+  // CTA pairs, one CTA per SM at most, all resident; a pair takes tiles round robin and runs
+  // them in order, and a tile waits only on tiles before it
+  const int pairs_max = di->sm_count / 2;
+  const int pairs = p.n_items < pairs_max ? p.n_items : pairs_max;
+  if (pairs < 1) return RA_ERR_DEVICE;
+  rf::ffn_kernel<<<2 * pairs, rf::NUM_THREADS, smem, stream>>>(mx, mw1, mz, mw2, p);
   return launch_status();
 }
 
