@@ -8,7 +8,7 @@
 // feedforward.  Y = gelu(X W1^T + b1) W2^T + b2 with X the block's attention output, heads side
 // by side per token; GELU in its exact form x Phi(x) (the pages name no activation).
 //
-// Work items (tiles of 128 rows x 256 columns), in this order, block after block:
+// Work items (tiles of 256 rows x 256 columns), in this order, block after block:
 //   GEMM 1 of block r: A = the attention output O [B][H][S][Dh] read in place (token rows of the
 //           block; K index = head * Dh + d), B = W1 [f][h], epi = bias + GELU, C = Z_u [B][c][f];
 //   GEMM 2 of block r: A = Z_u, B = W2 [h][f], epi = bias, C = the block's rows of Y [B][S][h].
@@ -29,9 +29,10 @@
 // step for 512 tensor cycles (64 B per clock, against 96 for a single CTA with 128 x 256 tiles).
 // Loads of both CTAs complete on the even CTA's barriers; the even CTA's one MMA thread issues
 // every MMA and commits to barriers in both CTAs.  Tiles are taken round robin by CTA pair.
-// CTA (256 threads): warps 0-3 epilogue (thread = output row = TMEM lane; the even CTA holds rows
-// 0-127 of the tile, the odd one rows 128-255), warp 4 TMA producer (6-stage ring of 32 KiB, no
-// multicast), warp 5 TMEM allocation (both CTAs) and, in the even CTA, the tcgen05.mma issue.
+// CTA (384 threads): warps 0-7 epilogue (thread = output row = TMEM lane; warps w and w + 4 share
+// lane quarter w, columns 0-127 and 128-255; the even CTA holds rows 0-127 of the tile, the odd one
+// rows 128-255), warp 8 TMA producer (6-stage ring of 32 KiB, no multicast), warp 9 TMEM
+// allocation (both CTAs) and, in the even CTA, the tcgen05.mma issue.
 // TMEM per CTA: two 128 x 256 fp32 accumulators, so a tile's epilogue runs under the next tile's
 // MMAs.
 #pragma once
@@ -43,8 +44,9 @@ namespace ffn {
 constexpr int BM = 256, BN = 256, BK = 64;   // tile of a CTA pair
 constexpr int HALF = 128;                     // rows of A and of B per CTA
 constexpr int NSTAGE = 6;
-constexpr int NUM_THREADS = 256;
-constexpr int WARP_TMA = 4, WARP_MMA = 5;
+constexpr int EPI_WARPS = 8;        // two per TMEM lane quarter, each taking half of the columns
+constexpr int NUM_THREADS = 384;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;   // warps 10-11 only complete the third warpgroup
 constexpr uint32_t TMEM_COLS = 512;
 
 struct Layout {
@@ -53,7 +55,8 @@ struct Layout {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = NSTAGE * STAGE_BYTES;
   // FULL: used in the even CTA (both CTAs' loads complete on it); EMPTY, ACC_FULL: in both CTAs
-  // (the even CTA's MMA commits to both); ACC_EMPTY: in the even CTA (4 warps of each CTA arrive)
+  // (the even CTA's MMA commits to both); ACC_EMPTY: in the even CTA (the epilogue warps of both
+  // CTAs arrive)
   static constexpr int B_FULL = 0, B_EMPTY = NSTAGE, B_ACC_FULL = 2 * NSTAGE, B_ACC_EMPTY = B_ACC_FULL + 2,
                        B_DRAIN = B_ACC_EMPTY + 2, NUM_BARS = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag
@@ -84,6 +87,10 @@ struct Tile {
   int mt, nt, b, tt;     // row tile in the block, column tile, batch entry, row tile in the entry
 };
 
+// Order of a block's tiles: the GEMM 1 tiles with the row tiles fastest (consecutive CTA pairs
+// share a weight slab in L2), then the GEMM 2 tiles the same way.  (Row tile by row tile, with each
+// row tile's GEMM 2 tiles right behind its GEMM 1 tiles, measured 24 % slower: the pairs in flight
+// then stream different weight slabs.)
 __device__ __forceinline__ Tile decode(int w, const Params& p) {
   Tile t;
   t.blk = w / p.per_block;
@@ -264,13 +271,16 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, int p
   drain_wait(bar(L::B_DRAIN), 0);
 }
 
-// ------------------------------------------------------------------ epilogue (128 threads per CTA)
+// ------------------------------------------------------------------ epilogue (256 threads per CTA)
 __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_t rank, int pair, int n_pairs,
                          volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
+  constexpr uint32_t NT = EPI_WARPS * 32;          // epilogue threads (named barrier 1)
   const int lane = threadIdx.x & 31;
-  const int quarter = threadIdx.x >> 5;            // warps 0-3: TMEM lanes 32 * quarter + lane
+  const int warp = threadIdx.x >> 5;
+  const int quarter = warp & 3;                    // TMEM lanes 32 * quarter + lane
+  const int col0 = (warp >> 2) * (BN / 2);         // this warp's half of the tile's columns
   const int r = static_cast<int>(rank) * HALF + quarter * 32 + lane;   // row within the pair's tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
   uint32_t acc_phases = 0;   // bit a: phase of accumulator a
@@ -279,7 +289,7 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_
     const Tile t = decode(w, p);
     const int acc = j & 1;
     // uniform outcomes across the four warps: the named barriers below need all of them
-    if (!named_bar_and(1, 128, mbar_wait(bar(L::B_ACC_FULL + acc), (acc_phases >> acc) & 1u, abort_flag))) return;
+    if (!named_bar_and(1, NT, mbar_wait(bar(L::B_ACC_FULL + acc), (acc_phases >> acc) & 1u, abort_flag))) return;
     acc_phases ^= 1u << acc;
     tc_fence_after();
     const int row_in_block = t.tt * BM + r;
@@ -293,7 +303,7 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_
       bool go = true;
       if (t.blk >= 2 && threadIdx.x == 0)
         go = wait_count(p.consumed + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT2 * (t.blk / 2)), abort_flag);
-      if (!named_bar_and(1, 128, go)) return;
+      if (!named_bar_and(1, NT, go)) return;
       crow = p.z + ((static_cast<long long>(t.u) * (p.MT / p.mt_per_b) + t.b) * p.c + row_in_block) * p.f;
       bias = p.b1;
       N = p.f;
@@ -304,13 +314,13 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_
       bias = p.b2;
       N = p.h;
     }
-    const int n_base = t.nt * BN;
+    const int n_base = t.nt * BN + col0;
 #pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
+    for (int ch = 0; ch < BN / 64; ++ch) {
       const int n0 = n_base + 32 * ch;
       if (n0 >= N) break;   // uniform: N is a multiple of 64
       uint32_t v[32];
-      tmem_ld32(lane_base + acc * BN + 32 * ch, v);
+      tmem_ld32(lane_base + acc * BN + col0 + 32 * ch, v);
       tmem_ld_wait();
       uint32_t pk[16];
 #pragma unroll
@@ -331,12 +341,12 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_
     }
     tc_fence_before();
     __syncwarp();
-    // 8 arrivals on the even CTA's barrier (4 warps of each CTA): the accumulator is free
+    // 2 * EPI_WARPS arrivals on the even CTA's barrier: the accumulator is free
     if (lane == 0) mbar_arrive_cluster(map_to_rank(bar(L::B_ACC_EMPTY + acc), 0));
     if (t.g == 1) {   // publish this CTA's half of the tile's Z columns
       fence_proxy_async_global();   // for the TMA (async proxy) reads that follow elsewhere
       __threadfence();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, NT);
       if (threadIdx.x == 0) signal_count(p.ready + t.u * p.MT + t.mt);
     }
   }
@@ -358,7 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       const bool acc_empty = i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1;
-      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 8 : 1);
+      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 2 * EPI_WARPS : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -381,7 +391,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp < 4) {
+  if (warp < EPI_WARPS) {
     epilogue(p, sbase, tmem, rank, pair, n_pairs, abort_flag);
   } else if (warp == WARP_TMA) {
     if ((threadIdx.x & 31) == 0) producer(&tm_x, &tm_w1, &tm_z, &tm_w2, p, sbase, rank, pair, n_pairs, abort_flag);
