@@ -7,8 +7,8 @@ Sources (page title, section):
         (close reading): §2.1 blockwise attention without materialising the s x s
         matrix; §3.1 a query block against a group of key/value blocks may be computed
         in any order if each block's statistics are combined with rescaling; §3.2 the
-        ring; §3.5 Algorithm 1 and its 4-device walk-through (round 1 uses the own
-        block, round 2 on device 0 uses block 3); summary: the result equals global
+        ring; §3.5 Algorithm 1 and its 4-device walk-through (the first ring step uses
+        the own block, the second on device 0 uses block 3); summary: the result equals global
         attention with no approximation.
   [HB]  "Ring Attention 与序列并行" (agent handbook): conceptual pseudocode — per ring
         step, attention of the local queries against the current K/V block, folded in
