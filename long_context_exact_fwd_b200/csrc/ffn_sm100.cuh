@@ -19,7 +19,9 @@
 //                  row tile m starts loading Z once all column tiles of its block are in;
 //   consumed[u][m] GEMM 2 tiles of row tile m whose MMAs have read Z; a GEMM 1 tile two blocks
 //                  later overwrites those rows only once every one of them has.
-// CTAs take items in that order from a global counter and run them in order, and an item only
+// CTA pairs take items in that order from a per-launch counter as they become free (a fixed round
+// robin let the pairs drift apart, since second-product tiles are four times longer, and left
+// second-product tiles waiting on first-product tiles taken late: 4 % slower), and an item only
 // waits on items before it, all taken by resident CTAs (one CTA per SM, grid <= SMs): every wait
 // ends.  Every wait is bounded all the same (RA_ERR_TIMEOUT, then the CTA unwinds).
 //
@@ -28,7 +30,8 @@
 // M = 256, N = 256 MMA per 16-wide K step runs on both SMs, so an SM brings in 32 KiB per 64-wide K
 // step for 512 tensor cycles (64 B per clock, against 96 for a single CTA with 128 x 256 tiles).
 // Loads of both CTAs complete on the even CTA's barriers; the even CTA's one MMA thread issues
-// every MMA and commits to barriers in both CTAs.  Tiles are taken round robin by CTA pair.
+// every MMA and commits to barriers in both CTAs.  The even CTA's producer takes the tile numbers
+// and hands each to every role of both CTAs through a ring of tile numbers in shared memory.
 // CTA (384 threads): warps 0-7 epilogue (thread = output row = TMEM lane; warps w and w + 4 share
 // lane quarter w, columns 0-127 and 128-255; the even CTA holds rows 0-127 of the tile, the odd one
 // rows 128-255), warp 8 TMA producer (6-stage ring of 32 KiB, no multicast), warp 9 TMEM
@@ -37,6 +40,7 @@
 // MMAs.
 #pragma once
 #include "ra_sm100.cuh"
+#include "ra_work.cuh"
 
 namespace ra {
 namespace ffn {
@@ -47,6 +51,7 @@ constexpr int NSTAGE = 6;
 constexpr int EPI_WARPS = 8;        // two per TMEM lane quarter, each taking half of the columns
 constexpr int NUM_THREADS = 384;
 constexpr int WARP_TMA = 8, WARP_MMA = 9;   // warps 10-11 only complete the third warpgroup
+constexpr int NITEM = 4;   // entries of the pair's ring of tile numbers
 constexpr uint32_t TMEM_COLS = 512;
 
 struct Layout {
@@ -57,10 +62,17 @@ struct Layout {
   // FULL: used in the even CTA (both CTAs' loads complete on it); EMPTY, ACC_FULL: in both CTAs
   // (the even CTA's MMA commits to both); ACC_EMPTY: in the even CTA (the epilogue warps of both
   // CTAs arrive)
+  // ITEM_FULL: in both CTAs (the even CTA's producer publishes each tile number to both);
+  // ITEM_EMPTY: in the even CTA (every reader of both CTAs arrives)
   static constexpr int B_FULL = 0, B_EMPTY = NSTAGE, B_ACC_FULL = 2 * NSTAGE, B_ACC_EMPTY = B_ACC_FULL + 2,
-                       B_DRAIN = B_ACC_EMPTY + 2, NUM_BARS = B_DRAIN + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag
-  static constexpr int BYTES = MISC_OFF + 16;
+                       B_DRAIN = B_ACC_EMPTY + 2, B_ITEM_FULL = B_DRAIN + 1, B_ITEM_EMPTY = B_ITEM_FULL + NITEM,
+                       NUM_BARS = B_ITEM_EMPTY + NITEM;
+  // readers of a tile number: the even CTA's MMA thread and its epilogue warps, the odd CTA's
+  // producer thread and its epilogue warps
+  static constexpr uint32_t ITEM_READERS = 2 + 2 * EPI_WARPS;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;   // TMEM base, abort flag, tile numbers
+  static constexpr int ITEMS_OFF = MISC_OFF + 8;
+  static constexpr int BYTES = ITEMS_OFF + 4 * NITEM;
   static constexpr int ALLOC = BYTES + 1024;                // room to align the base to 1024 B
 };
 static_assert(Layout::ALLOC <= 232448, "shared memory");
@@ -73,6 +85,7 @@ struct Params {
   int NT1, NT2;          // column tiles of GEMM 1 (f) and GEMM 2 (h)
   int per_block;         // MT * (NT1 + NT2)
   int n_items;           // nblocks * per_block
+  int work_slot;         // this launch's work counter
   const float* b1;       // [f]
   const float* b2;       // [h]
   __nv_bfloat16* z;      // [2][B][c][f] hidden activations (one buffer when nblocks == 1)
@@ -180,16 +193,102 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
                : "memory");
 }
 
+// Tile numbers of the pair.  The even CTA's producer takes them from the launch's work counter
+// (dynamic: a pair that finishes early takes the next tile, so the pairs do not drift apart the
+// way a fixed round robin of tiles of unequal length makes them) and writes each into the same
+// ring entry of both CTAs.  Readers wait on their own CTA's ITEM_FULL with cluster-scope acquire
+// and arrive on the even CTA's ITEM_EMPTY.
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 0; it != 0xffffffffu; ++it) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    if ((it & 127u) == 127u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > RA_WAIT_TIMEOUT_NS) break;
+    }
+  }
+  *abort_flag = 1;
+  record_status(RA_ERR_TIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+struct PairItems {
+  uint32_t sbase;
+  int k = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ uint32_t bar(int i) const { return sbase + Layout::BAR_OFF + 8u * i; }
+  __device__ __forceinline__ uint32_t slot() const { return sbase + Layout::ITEMS_OFF + 4u * k; }
+  __device__ __forceinline__ void advance() {
+    if (++k == NITEM) {
+      k = 0;
+      ph ^= 1u;
+    }
+  }
+  // even CTA's producer: publish `item` to both CTAs once every reader has read the entry's last
+  __device__ __forceinline__ bool push(int item, volatile int* abort_flag) {
+    if (!mbar_wait(bar(Layout::B_ITEM_EMPTY + k), ph ^ 1u, abort_flag)) return false;
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(slot()), "r"(static_cast<uint32_t>(item)) : "memory");
+    st_cluster_u32(map_to_rank(slot(), 1), static_cast<uint32_t>(item));
+    mbar_arrive(bar(Layout::B_ITEM_FULL + k));
+    mbar_arrive_cluster(map_to_rank(bar(Layout::B_ITEM_FULL + k), 1));   // release: the store above first
+    advance();
+    return true;
+  }
+  // one reading thread (arrives once)
+  __device__ __forceinline__ bool pop(int& item, volatile int* abort_flag) {
+    if (!mbar_wait_acq_cluster(bar(Layout::B_ITEM_FULL + k), ph, abort_flag)) return false;
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(slot()) : "memory");
+    item = static_cast<int>(v);
+    mbar_arrive_cluster(map_to_rank(bar(Layout::B_ITEM_EMPTY + k), 0));
+    advance();
+    return true;
+  }
+  // a whole warp reads, lane 0 arrives once; uniform outcome
+  __device__ __forceinline__ bool pop_warp(int& item, volatile int* abort_flag) {
+    if (!__all_sync(0xffffffffu, mbar_wait_acq_cluster(bar(Layout::B_ITEM_FULL + k), ph, abort_flag))) return false;
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(slot()) : "memory");
+    item = static_cast<int>(v);
+    __syncwarp();
+    if ((threadIdx.x & 31u) == 0u) mbar_arrive_cluster(map_to_rank(bar(Layout::B_ITEM_EMPTY + k), 0));
+    advance();
+    return true;
+  }
+};
+
 // ------------------------------------------------------------------ producer (1 thread per CTA)
 __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, const CUtensorMap* tm_z,
-                         const CUtensorMap* tm_w2, const Params& p, uint32_t sbase, uint32_t rank, int pair,
-                         int n_pairs, volatile int* abort_flag) {
+                         const CUtensorMap* tm_w2, const Params& p, uint32_t sbase, uint32_t rank,
+                         volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   int stage = 0;
   uint32_t phase = 0, issued = 0, issued_parity = 0;
   bool ok = true;
-  for (int w = pair; w < p.n_items && ok; w += n_pairs) {
+  PairItems items{sbase};
+  int w = rank == 0 ? work_fetch(p.work_slot) : 0;
+  for (;;) {
+    if (rank == 0 ? !items.push(w, abort_flag) : !items.pop(w, abort_flag)) {
+      ok = false;
+      break;
+    }
+    if (w >= p.n_items) break;
+    const int w_next = rank == 0 ? work_fetch(p.work_slot) : 0;   // in flight while this tile's loads issue
     const Tile t = decode(w, p);
     const int r = p.r0 + t.blk;
     const int K = t.g == 1 ? p.h : p.f;
@@ -220,7 +319,10 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, cons
         phase ^= 1u;
       }
     }
+    if (!ok) break;
+    w = w_next;
   }
+  work_done(p.work_slot);   // each CTA once (the odd one after reading the end marker)
   if (!ok && rank == 0) {   // let every copy the pair started land (they count on these barriers)
     for (int s = 0; s < NSTAGE; ++s)
       if (issued & (1u << s)) drain_wait(bar(L::B_FULL + s), (issued_parity >> s) & 1u);
@@ -228,8 +330,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, cons
 }
 
 // ------------------------------------------------------------------ MMA issuer (1 thread, even CTA)
-__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, int pair, int n_pairs,
-                           volatile int* abort_flag) {
+__device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   auto both = [&](int i) {   // commit to barrier i of each CTA
@@ -240,8 +341,10 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, int p
   int stage = 0;
   uint32_t phase = 0;
   uint32_t acc_phases = 0;   // bit a: phase of accumulator a
-  int j = 0;
-  for (int w = pair; w < p.n_items; w += n_pairs, ++j) {
+  PairItems items{sbase};
+  for (int j = 0;; ++j) {
+    int w;
+    if (!items.pop(w, abort_flag) || w >= p.n_items) break;
     const Tile t = decode(w, p);
     const int K = t.g == 1 ? p.h : p.f;
     const int acc = j & 1;
@@ -272,8 +375,7 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, int p
 }
 
 // ------------------------------------------------------------------ epilogue (256 threads per CTA)
-__device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_t rank, int pair, int n_pairs,
-                         volatile int* abort_flag) {
+__device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_t rank, volatile int* abort_flag) {
   using L = Layout;
   auto bar = [&](int i) { return sbase + L::BAR_OFF + 8u * i; };
   constexpr uint32_t NT = EPI_WARPS * 32;          // epilogue threads (named barrier 1)
@@ -284,8 +386,12 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_
   const int r = static_cast<int>(rank) * HALF + quarter * 32 + lane;   // row within the pair's tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
   uint32_t acc_phases = 0;   // bit a: phase of accumulator a
-  int j = 0;
-  for (int w = pair; w < p.n_items; w += n_pairs, ++j) {
+  PairItems items{sbase};
+  for (int j = 0;; ++j) {
+    int w;
+    // uniform outcome across the epilogue warps (the named barriers below need all of them)
+    const bool got = items.pop_warp(w, abort_flag);
+    if (!named_bar_and(1, NT, got && w < p.n_items)) return;
     const Tile t = decode(w, p);
     const int acc = j & 1;
     // uniform outcomes across the four warps: the named barriers below need all of them
@@ -364,11 +470,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const int warp = threadIdx.x >> 5;
   const uint32_t rank = cluster_rank();
-  const int pair = static_cast<int>(blockIdx.x >> 1), n_pairs = static_cast<int>(gridDim.x >> 1);
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       const bool acc_empty = i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1;
-      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 2 * EPI_WARPS : 1);
+      const bool item_empty = i >= L::B_ITEM_EMPTY && i < L::B_ITEM_EMPTY + NITEM;
+      mbar_init(sbase + L::BAR_OFF + 8u * i, acc_empty ? 2 * EPI_WARPS : (item_empty ? L::ITEM_READERS : 1));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -392,12 +498,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp < EPI_WARPS) {
-    epilogue(p, sbase, tmem, rank, pair, n_pairs, abort_flag);
+    epilogue(p, sbase, tmem, rank, abort_flag);
   } else if (warp == WARP_TMA) {
-    if ((threadIdx.x & 31) == 0) producer(&tm_x, &tm_w1, &tm_z, &tm_w2, p, sbase, rank, pair, n_pairs, abort_flag);
+    if ((threadIdx.x & 31) == 0) producer(&tm_x, &tm_w1, &tm_z, &tm_w2, p, sbase, rank, abort_flag);
     __syncwarp();
   } else if (warp == WARP_MMA) {
-    if (rank == 0 && (threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, pair, n_pairs, abort_flag);
+    if (rank == 0 && (threadIdx.x & 31) == 0) mma_issuer(p, sbase, tmem, abort_flag);
     __syncwarp();
   }
 

@@ -729,6 +729,7 @@ int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nbloc
   if (per_block * nblocks > INT_MAX) return RA_ERR_SHAPE;
   p.per_block = static_cast<int>(per_block);
   p.n_items = static_cast<int>(per_block * nblocks);
+  p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.b1 = b1;
   p.b2 = b2;
   p.z = static_cast<__nv_bfloat16*>(workspace);
