@@ -228,11 +228,12 @@ RA_API int ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, co
 RA_API size_t ring_attn_bwd_noalloc_max_bytes(void);
 
 /*
- * ring_attn_ffn_workspace_size -- bytes of device workspace the blockwise feedforward needs: two
- * ring blocks' hidden activations, bf16 [2][B][S / D][f] (block r + 1's first product runs while
- * block r's second drains), then 4 * B * ceil((S / D) / 256) 32-bit dependency counters, each
- * region rounded up to 256 bytes.  Independent of D for a given block size: the activation alive
- * is two blocks', never the sequence's.  Returns 0 for invalid sizes.
+ * ring_attn_ffn_workspace_size -- bytes of device workspace the blockwise feedforward needs:
+ * nbuf = min(3, D) ring blocks' hidden activations, bf16 [nbuf][B][S / D][f] (block r + 1's first
+ * product runs before block r's second, so that neither waits on the other's last tiles), then
+ * 2 * nbuf * B * ceil((S / D) / 256) 32-bit dependency counters, each region rounded up to 256
+ * bytes.  Bounded by three blocks for a given block size: the activation alive is at most three
+ * blocks', never the sequence's.  Returns 0 for invalid sizes.
  */
 RA_API size_t ring_attn_ffn_workspace_size(int B, int S, int D, int f);
 
@@ -271,9 +272,10 @@ RA_API int ring_attn_ffn_block(const void* o, int B, int H, int S, int Dh, int D
 
 /*
  * ring_attn_ffn_fwd -- the feedforward of every ring block r = 0 .. D-1, in that order, in one
- * persistent launch: block r + 1's first product overlaps block r's second, and the two
- * block-sized activation buffers of the workspace alternate, so at most two blocks' hidden
- * activations are alive, whatever the sequence length.  Arguments and errors as
+ * persistent launch, in the order: first product of block 0, then for r = 1 .. D-1 the first
+ * product of block r and the second of block r - 1, then the second of block D-1.  The
+ * block-sized activation buffers of the workspace rotate (block r uses buffer r mod min(3, D)), so
+ * at most three blocks' hidden activations are alive, whatever the sequence length.  Arguments and errors as
  * ring_attn_ffn_block (without r).
  */
 RA_API int ring_attn_ffn_fwd(const void* o, int B, int H, int S, int Dh, int D, const void* w1, const float* b1,

@@ -8,17 +8,21 @@
 // feedforward.  Y = gelu(X W1^T + b1) W2^T + b2 with X the block's attention output, heads side
 // by side per token; GELU in its exact form x Phi(x) (the pages name no activation).
 //
-// Work items (tiles of 256 rows x 256 columns), in this order, block after block:
+// Work items (tiles of 256 rows x 256 columns):
 //   GEMM 1 of block r: A = the attention output O [B][H][S][Dh] read in place (token rows of the
 //           block; K index = head * Dh + d), B = W1 [f][h], epi = bias + GELU, C = Z_u [B][c][f];
-//   GEMM 2 of block r: A = Z_u, B = W2 [h][f], epi = bias, C = the block's rows of Y [B][S][h].
-// Z_u (u = block index in the launch mod 2) are two block-sized hidden activations in the
-// caller's workspace, so block r + 1's GEMM 1 runs while block r's GEMM 2 drains.  Dependencies,
-// through per-row-tile counters in the workspace (cleared before the launch):
+//   GEMM 2 of block r: A = Z_u, B = W2 [h][f], epi = bias, C = the block's rows of Y [B][S][h];
+// in the order GEMM 1 of block 0, then for r = 1, 2, ...: GEMM 1 of block r, GEMM 2 of block r - 1,
+// and last GEMM 2 of the final block.  Z_u (u = block index in the launch mod nbuf, nbuf =
+// min(3, D)) are block-sized hidden activations in the caller's workspace.  Dependencies, through
+// per-row-tile counters in the workspace (cleared before the launch):
 //   ready[u][m]    GEMM 1 tiles of row tile m that have stored their Z columns; a GEMM 2 tile of
 //                  row tile m starts loading Z once all column tiles of its block are in;
-//   consumed[u][m] GEMM 2 tiles of row tile m whose MMAs have read Z; a GEMM 1 tile two blocks
+//   consumed[u][m] GEMM 2 tiles of row tile m whose MMAs have read Z; a GEMM 1 tile nbuf blocks
 //                  later overwrites those rows only once every one of them has.
+// The lag puts a whole segment of other tiles between each tile and what it waits for: a block's
+// GEMM 2 waits on GEMM 1 tiles taken a segment earlier, and with three buffers a GEMM 1 tile
+// waits on GEMM 2 tiles two segments back.
 // CTA pairs take items in that order from a per-launch counter as they become free (a fixed round
 // robin let the pairs drift apart, since second-product tiles are four times longer, and left
 // second-product tiles waiting on first-product tiles taken late: 4 % slower), and an item only
@@ -85,13 +89,14 @@ struct Params {
   int NT1, NT2;          // column tiles of GEMM 1 (f) and GEMM 2 (h)
   int per_block;         // MT * (NT1 + NT2)
   int n_items;           // nblocks * per_block
+  int nbuf;              // hidden-activation buffers: min(3, D)
   int work_slot;         // this launch's work counter
   const float* b1;       // [f]
   const float* b2;       // [h]
-  __nv_bfloat16* z;      // [2][B][c][f] hidden activations (one buffer when nblocks == 1)
+  __nv_bfloat16* z;      // [nbuf][B][c][f] hidden activations
   __nv_bfloat16* y;      // [B][S][h]
-  unsigned* ready;       // [2][MT]
-  unsigned* consumed;    // [2][MT]
+  unsigned* ready;       // [nbuf][MT]
+  unsigned* consumed;    // [nbuf][MT]
 };
 
 struct Tile {
@@ -100,20 +105,34 @@ struct Tile {
   int mt, nt, b, tt;     // row tile in the block, column tile, batch entry, row tile in the entry
 };
 
-// Order of a block's tiles: the GEMM 1 tiles with the row tiles fastest (consecutive CTA pairs
-// share a weight slab in L2), then the GEMM 2 tiles the same way.  (Row tile by row tile, with each
-// row tile's GEMM 2 tiles right behind its GEMM 1 tiles, measured 24 % slower: the pairs in flight
-// then stream different weight slabs.)
+// Item w -> tile.  Segments: GEMM 1 of block 0; then (GEMM 1 of block k, GEMM 2 of block k - 1)
+// for k = 1 .. nblocks - 1; then GEMM 2 of the last block.  Inside a segment the row tiles go
+// fastest (consecutive CTA pairs share a weight slab in L2).  (Row tile by row tile, with each row
+// tile's GEMM 2 tiles right behind its GEMM 1 tiles, measured 24 % slower: the pairs in flight then
+// stream different weight slabs.)
 __device__ __forceinline__ Tile decode(int w, const Params& p) {
+  const int s1 = p.MT * p.NT1, s2 = p.MT * p.NT2;
   Tile t;
-  t.blk = w / p.per_block;
-  int idx = w - t.blk * p.per_block;
-  t.u = t.blk & 1;
-  t.g = 1;
-  if (idx >= p.MT * p.NT1) {
-    idx -= p.MT * p.NT1;
-    t.g = 2;
+  int idx;
+  if (w < s1) {
+    t.blk = 0;
+    t.g = 1;
+    idx = w;
+  } else {
+    const int v = w - s1;
+    const int q = v / (s1 + s2);
+    const int off = v - q * (s1 + s2);
+    if (q < p.nblocks - 1 && off < s1) {
+      t.blk = q + 1;
+      t.g = 1;
+      idx = off;
+    } else {
+      t.blk = q;
+      t.g = 2;
+      idx = q < p.nblocks - 1 ? off - s1 : off;
+    }
   }
+  t.u = t.blk % p.nbuf;
   t.mt = idx % p.MT;
   t.nt = idx / p.MT;
   t.b = t.mt / p.mt_per_b;
@@ -294,7 +313,7 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, cons
     const int K = t.g == 1 ? p.h : p.f;
     const int row = t.tt * BM + rank * HALF;   // this CTA's rows of the tile, within the batch entry
     if (t.g == 2) {   // every column tile of this row tile's hidden activation is stored (both CTAs)
-      if (!wait_count(p.ready + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT1 * (t.blk / 2 + 1)), abort_flag)) {
+      if (!wait_count(p.ready + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT1 * (t.blk / p.nbuf + 1)), abort_flag)) {
         ok = false;
         break;
       }
@@ -404,11 +423,11 @@ __device__ void epilogue(const Params& p, uint32_t sbase, uint32_t tmem, uint32_
     const float* bias;
     int N;
     if (t.g == 1) {
-      // Z_u rows of this row tile are overwritten only once the GEMM 2 tiles of the block two
+      // Z_u rows of this row tile are overwritten only once the GEMM 2 tiles of the block nbuf
       // before have read them
       bool go = true;
-      if (t.blk >= 2 && threadIdx.x == 0)
-        go = wait_count(p.consumed + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT2 * (t.blk / 2)), abort_flag);
+      if (t.blk >= p.nbuf && threadIdx.x == 0)
+        go = wait_count(p.consumed + t.u * p.MT + t.mt, static_cast<unsigned>(2 * p.NT2 * (t.blk / p.nbuf)), abort_flag);
       if (!named_bar_and(1, NT, go)) return;
       crow = p.z + ((static_cast<long long>(t.u) * (p.MT / p.mt_per_b) + t.b) * p.c + row_in_block) * p.f;
       bias = p.b1;

@@ -669,15 +669,17 @@ namespace {
 // dependency counters ([2][MT] ready, [2][MT] consumed), each region 256-byte aligned.
 struct FfnWorkspace {
   size_t z_bytes, ctr_bytes, total;
-  int mt;
+  int mt;     // row tiles of 256 per block: B * ceil(c / 256)
+  int nbuf;   // block-sized hidden-activation buffers: min(3, D)
 };
 
 FfnWorkspace ffn_workspace(int B, int S, int D, int f) {
   FfnWorkspace w;
   const int c = S / D;
   w.mt = B * ((c + ra::ffn::BM - 1) / ra::ffn::BM);
-  w.z_bytes = align256(2 * static_cast<size_t>(B) * c * f * 2);
-  w.ctr_bytes = align256(static_cast<size_t>(4) * w.mt * sizeof(unsigned));
+  w.nbuf = D < 3 ? D : 3;
+  w.z_bytes = align256(static_cast<size_t>(w.nbuf) * B * c * f * 2);
+  w.ctr_bytes = align256(static_cast<size_t>(2 * w.nbuf) * w.mt * sizeof(unsigned));
   w.total = w.z_bytes + w.ctr_bytes;
   return w;
 }
@@ -729,20 +731,21 @@ int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nbloc
   if (per_block * nblocks > INT_MAX) return RA_ERR_SHAPE;
   p.per_block = static_cast<int>(per_block);
   p.n_items = static_cast<int>(per_block * nblocks);
+  p.nbuf = ws.nbuf;
   p.work_slot = static_cast<int>(di->next_work_slot.fetch_add(1) % ra::WORK_SLOTS);
   p.b1 = b1;
   p.b2 = b2;
   p.z = static_cast<__nv_bfloat16*>(workspace);
   p.y = static_cast<__nv_bfloat16*>(y);
   p.ready = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + ws.z_bytes);
-  p.consumed = p.ready + 2 * p.MT;
+  p.consumed = p.ready + ws.nbuf * p.MT;
   CUtensorMap mx, mw1, mz, mw2;
   // each CTA of a pair loads 128 rows of A and 128 of the tile's 256 B rows per K step
   if ((st = make_map(&mx, o, static_cast<long long>(B) * H, S, Dh, rf::HALF)) != RA_OK) return st;
   if ((st = make_map(&mw1, w1, 1, f, p.h, rf::HALF)) != RA_OK) return st;
-  if ((st = make_map(&mz, workspace, 2ll * B, p.c, f, rf::HALF)) != RA_OK) return st;
+  if ((st = make_map(&mz, workspace, static_cast<long long>(ws.nbuf) * B, p.c, f, rf::HALF)) != RA_OK) return st;
   if ((st = make_map(&mw2, w2, 1, p.h, f, rf::HALF)) != RA_OK) return st;
-  const cudaError_t me = cudaMemsetAsync(p.ready, 0, 4 * static_cast<size_t>(p.MT) * sizeof(unsigned), stream);
+  const cudaError_t me = cudaMemsetAsync(p.ready, 0, ws.ctr_bytes, stream);
   if (me != cudaSuccess) return cuda_fail(static_cast<int>(me), "cudaMemsetAsync(ffn counters)");
   constexpr int smem = rf::Layout::ALLOC;
   if (!di->ffn_attr) {
@@ -750,8 +753,8 @@ int ffn_run(const void* o, int B, int H, int S, int Dh, int D, int r0, int nbloc
     if (e != cudaSuccess) return cuda_fail(static_cast<int>(e), "cudaFuncSetAttribute(ffn smem)");
     di->ffn_attr = true;
   }
-  // CTA pairs, one CTA per SM at most, all resident; a pair takes tiles round robin and runs
-  // them in order, and a tile waits only on tiles before it
+  // CTA pairs, one CTA per SM at most, all resident; pairs take tiles in order from the launch's
+  // counter, and a tile waits only on tiles before it
   const int pairs_max = di->sm_count / 2;
   const int pairs = p.n_items < pairs_max ? p.n_items : pairs_max;
   if (pairs < 1) return RA_ERR_DEVICE;

@@ -111,14 +111,15 @@ def test_ffn_argument_errors(ra):
     assert f(*args(S=301)) == ra.RA_ERR_SHAPE       # uneven ring split
     assert f(*args(b1=260)) == ra.RA_ERR_ALIGN
     assert f(*args(ws=0)) == ra.RA_ERR_WORKSPACE
-    assert f(*args(wsb=2 * 100 * 256 * 2)) == ra.RA_ERR_WORKSPACE   # no room for the counters
-    # two blocks' hidden activations, bf16 [2][B][S/D][f], then 4 * (B * ceil(c / 256)) counters
-    # (one per 256-row tile of a CTA pair), each region rounded up to 256 bytes
+    assert f(*args(wsb=3 * 100 * 256 * 2)) == ra.RA_ERR_WORKSPACE   # no room for the counters
+    # min(3, D) blocks' hidden activations, bf16 [nbuf][B][S/D][f], then 2 * nbuf * (B * ceil(c / 256))
+    # counters (one per 256-row tile of a CTA pair and buffer), each region rounded up to 256 bytes
     r256 = lambda x: (x + 255) // 256 * 256
-    assert ra.ffn_workspace_bytes(1, 300, 3, 256) == r256(2 * 100 * 256 * 2) + r256(4 * 1 * 4)
-    assert ra.ffn_workspace_bytes(2, 300, 3, 64) == r256(2 * 2 * 100 * 64 * 2) + r256(4 * 2 * 4)
+    assert ra.ffn_workspace_bytes(1, 300, 3, 256) == r256(3 * 100 * 256 * 2) + r256(6 * 1 * 4)
+    assert ra.ffn_workspace_bytes(2, 300, 3, 64) == r256(3 * 2 * 100 * 64 * 2) + r256(6 * 2 * 4)
     assert ra.ffn_workspace_bytes(1, 1024, 2, 64) == r256(2 * 512 * 64 * 2) + r256(4 * 2 * 4)
-    assert ra.ffn_workspace_bytes(64, 65536, 1, 64) == r256(2 * 64 * 65536 * 64 * 2) + r256(4 * 64 * 256 * 4)
+    assert ra.ffn_workspace_bytes(64, 65536, 1, 64) == r256(64 * 65536 * 64 * 2) + r256(2 * 64 * 256 * 4)
+    assert ra.ffn_workspace_bytes(1, 8192, 8, 1024) == r256(3 * 1024 * 1024 * 2) + r256(6 * 4 * 4)
     assert ra.ffn_workspace_bytes(1, 300, 7, 256) == 0
 
 
