@@ -38,7 +38,9 @@
 // and hands each to every role of both CTAs through a ring of tile numbers in shared memory.
 // CTA (384 threads): warps 0-7 epilogue (thread = output row = TMEM lane; warps w and w + 4 share
 // lane quarter w, columns 0-127 and 128-255; the even CTA holds rows 0-127 of the tile, the odd one
-// rows 128-255), warp 8 TMA producer (6-stage ring of 32 KiB, no multicast), warp 9 TMEM
+// rows 128-255), warp 8 TMA producer (3-stage ring of 64 KiB: 128-wide K steps, so the MMA
+// thread waits and commits once per 8 MMAs; 3 % faster than 64-wide steps in 6 stages; no
+// multicast), warp 9 TMEM
 // allocation (both CTAs) and, in the even CTA, the tcgen05.mma issue.
 // TMEM per CTA: two 128 x 256 fp32 accumulators, so a tile's epilogue runs under the next tile's
 // MMAs.
@@ -49,9 +51,9 @@
 namespace ra {
 namespace ffn {
 
-constexpr int BM = 256, BN = 256, BK = 64;   // tile of a CTA pair
+constexpr int BM = 256, BN = 256, BK = 128;   // tile of a CTA pair, K step of a stage
 constexpr int HALF = 128;                     // rows of A and of B per CTA
-constexpr int NSTAGE = 6;
+constexpr int NSTAGE = 3;
 constexpr int EPI_WARPS = 8;        // two per TMEM lane quarter, each taking half of the columns
 constexpr int NUM_THREADS = 384;
 constexpr int WARP_TMA = 8, WARP_MMA = 9;   // warps 10-11 only complete the third warpgroup
@@ -59,8 +61,9 @@ constexpr int NITEM = 4;   // entries of the pair's ring of tile numbers
 constexpr uint32_t TMEM_COLS = 512;
 
 struct Layout {
-  static constexpr int A_BYTES = HALF * BK * 2;          // 16 KB: this CTA's 128 rows x 128 B
-  static constexpr int B_BYTES = HALF * BK * 2;          // 16 KB: this CTA's 128 of the 256 B rows
+  static constexpr int SUB_BYTES = HALF * 64 * 2;        // 128 rows x 64 columns (128 B, swizzled)
+  static constexpr int A_BYTES = (BK / 64) * SUB_BYTES;  // 32 KB: this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BK / 64) * SUB_BYTES;  // 32 KB: this CTA's 128 of the 256 B rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = NSTAGE * STAGE_BYTES;
   // FULL: used in the even CTA (both CTAs' loads complete on it); EMPTY, ACC_FULL: in both CTAs
@@ -323,13 +326,20 @@ __device__ void producer(const CUtensorMap* tm_x, const CUtensorMap* tm_w1, cons
       if (!mbar_wait(bar(L::B_EMPTY + stage), phase ^ 1u, abort_flag)) { ok = false; break; }
       const uint32_t st = sbase + stage * L::STAGE_BYTES;
       const uint32_t full = map_to_rank(bar(L::B_FULL + stage), 0);   // the even CTA's barrier
-      if (rank == 0) mbar_arrive_expect_tx(bar(L::B_FULL + stage), 2 * L::STAGE_BYTES);   // both CTAs' bytes
-      if (t.g == 1) {
-        tma_load_3d_pair(tm_x, st, full, k0 % p.Dh, r * p.c + row, t.b * p.H + k0 / p.Dh);
-        tma_load_3d_pair(tm_w1, st + L::A_BYTES, full, k0, t.nt * BN + rank * HALF, 0);
-      } else {
-        tma_load_3d_pair(tm_z, st, full, k0, row, t.u * (p.MT / p.mt_per_b) + t.b);
-        tma_load_3d_pair(tm_w2, st + L::A_BYTES, full, k0, t.nt * BN + rank * HALF, 0);
+      // 64-column sub-steps (the last step of a K that is an odd multiple of 64 has one: a load
+      // past the end of the attention output's heads would read the next batch entry's)
+      const int nsub = K - k0 >= BK ? BK / 64 : 1;
+      if (rank == 0) mbar_arrive_expect_tx(bar(L::B_FULL + stage), 4 * nsub * L::SUB_BYTES);   // both CTAs' bytes
+      for (int j = 0; j < nsub; ++j) {
+        const int kj = k0 + 64 * j;
+        const uint32_t sj = st + j * L::SUB_BYTES;
+        if (t.g == 1) {
+          tma_load_3d_pair(tm_x, sj, full, kj % p.Dh, r * p.c + row, t.b * p.H + kj / p.Dh);
+          tma_load_3d_pair(tm_w1, sj + L::A_BYTES, full, kj, t.nt * BN + rank * HALF, 0);
+        } else {
+          tma_load_3d_pair(tm_z, sj, full, kj, row, t.u * (p.MT / p.mt_per_b) + t.b);
+          tma_load_3d_pair(tm_w2, sj + L::A_BYTES, full, kj, t.nt * BN + rank * HALF, 0);
+        }
       }
       issued |= 1u << stage;
       issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -376,10 +386,14 @@ __device__ void mma_issuer(const Params& p, uint32_t sbase, uint32_t tmem, volat
       if (!mbar_wait(bar(L::B_FULL + stage), phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = sbase + stage * L::STAGE_BYTES, sb = sa + L::A_BYTES;
+      const int nk = K - k0 >= BK ? BK / 16 : 4;   // 16-wide MMAs of this step (4 on a 64-wide tail)
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk)
-        umma_ss_pair(d, sdesc_sw128(sa + kk * 32, 16, 1024), sdesc_sw128(sb + kk * 32, 16, 1024), IDESC,
-                     (k0 > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * L::SUB_BYTES + (kk & 3) * 32;
+        if (kk < nk)
+          umma_ss_pair(d, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024), IDESC,
+                       (k0 > 0 || kk > 0) ? 1u : 0u);
+      }
       both(L::B_EMPTY + stage);   // the stage is free in both CTAs once these MMAs have read it
       if (++stage == NSTAGE) {
         stage = 0;
