@@ -101,7 +101,7 @@ def _peaks():
 KERNEL_SOURCES = {
     "fwd_kernel": ("fwd_sm100.cuh", "ra_sm100.cuh", "ra_schedule.h", "ra_work.cuh", "ring_attn.cu"),
     "bwd_kernel": ("bwd_sm100.cuh", "ra_sm100.cuh", "ra_schedule.h", "ra_work.cuh", "ring_attn.cu"),
-    "ffn_kernel": ("ffn_sm100.cuh", "ra_sm100.cuh", "ra_work.cuh", "ring_attn.cu"),
+    "ffn_kernel": ("ffn_sm100.cuh", "ffn_host.cuh", "ra_sm100.cuh", "ra_work.cuh", "ring_attn.cu"),
 }
 
 
