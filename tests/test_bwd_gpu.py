@@ -47,7 +47,8 @@ def test_s16k_fwd_bwd_on_oracle_heads(ra):
 
 
 BWD_SHAPES = [(1, 2, 256, 128, 2), (1, 2, 300, 128, 3), (2, 1, 129, 128, 3), (1, 1, 1000, 128, 8),
-              (1, 2, 2048, 128, 4), (1, 1, 1, 128, 1), (1, 3, 640, 128, 5)]
+              (1, 2, 2048, 128, 4), (1, 1, 1, 128, 1), (1, 3, 640, 128, 5),
+              (1, 1, 64, 128, 64)]   # D = S: every ring block one token
 
 
 @pytest.mark.parametrize("causal", [False, True])

@@ -29,10 +29,11 @@ def _weights(h, f, seed):
 # (B, H, S, Dh, D, f): ragged blocks (c = 100, 125 < 128 rows), a partial last N tile
 # (f = 320, h = 192), both head dims; K = h or f an odd multiple of 64 (a 64-wide last K step),
 # with two batch entries where the first product's last step ends at a batch entry's last head;
-# one block (one activation buffer) and seven blocks (three buffers, reused up to twice)
+# one block (one activation buffer) and seven blocks (three buffers, reused up to twice); D = S
+# (one-token blocks)
 FFN_SHAPES = [(1, 2, 256, 64, 2, 256), (2, 1, 300, 128, 3, 320), (1, 4, 1000, 64, 8, 1024),
               (1, 3, 384, 64, 3, 512), (2, 2, 512, 128, 4, 1024), (2, 3, 256, 64, 2, 192),
-              (1, 2, 256, 64, 1, 256), (1, 1, 1792, 128, 7, 256)]
+              (1, 2, 256, 64, 1, 256), (1, 1, 1792, 128, 7, 256), (1, 1, 64, 128, 64, 128)]
 
 
 @pytest.mark.parametrize("B,H,S,Dh,D,f", FFN_SHAPES)

@@ -96,6 +96,7 @@ SHAPES = [  # (B, H, S, Dh, D): tiles, ragged tails, blocks smaller than a tile
     (1, 1, 1, 128, 1), (1, 2, 100, 128, 4), (2, 2, 128, 128, 2), (1, 2, 129, 128, 3), (1, 3, 255, 128, 5),
     (1, 2, 256, 128, 8), (1, 2, 257, 128, 1), (2, 1, 384, 128, 3), (1, 2, 1000, 128, 8), (1, 1, 2125, 128, 5),
     (1, 2, 777, 64, 7), (2, 2, 512, 64, 4), (1, 1, 64, 64, 2),
+    (1, 2, 64, 128, 64),   # D = S: every ring block one token
 ]
 
 
